@@ -1,0 +1,520 @@
+"""WBMM benchmark on B200: TFLOP/s, HBM GB/s and fraction of roofline.
+
+One step is one pass of the operator's hot path over one batch of seeded
+synthetic input.  Default workload (the training step): B128 C256 28x28, w=14,
+bf16 -- forward y = WBMM(x; T), then the backward dX = M^T dY and the table
+gradient dT, all through the C ABI.  Other workloads (--workload): fwd
+(B64 C128 56x56 w14), sweep7 / sweep14 / sweep28 (B32 C256 112x112), cached
+(B8 C96 224x224 w14, cached matrices + 3x3 mixing).
+
+Multi-GPU (torchrun): every rank owns its own block of channels with the
+per-GPU workload above (weak scaling); channels are independent, so the hot
+path has no collective.  Timing is device time (CUDA events) with a barrier on
+both sides, max over ranks.
+
+--impl reference runs the fp64 CPU oracle on the host cores instead (bounded
+sample per step); it is the slow baseline the driver divides by.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+import torch.distributed as dist
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "WBMM fwd/bwd TFLOP/s, HBM GB/s and % of roofline at w=14 bf16 on 1 B200"
+L2_BYTES = 126 * 2 ** 20
+
+WORKLOADS = {
+    "train": "train_bf16",
+    "fwd": "fwd_bf16",
+    "sweep7": "sweep_w7",
+    "sweep14": "sweep_w14",
+    "sweep28": "sweep_w28",
+    "cached": "hires_cached_dw",
+}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+# ------------------------------------------------------------ workload math
+
+def step_flops(wl):
+    n = wl.B * wl.C * wl.H * wl.W
+    f = 2.0 * n * wl.d
+    if wl.kind == "train":
+        return 3 * f
+    if wl.kind == "cached_dw":
+        return f + 18.0 * n
+    return f
+
+
+def step_bytes(wl):
+    """Algorithmic bytes: each tensor of the step read or written once."""
+    e = 2 if wl.dtype == "bf16" else 4
+    m = wl.B * wl.C * wl.H * wl.W * e
+    tbl = wl.C * wl.t * e
+    if wl.kind == "train":
+        return 5 * m + tbl + wl.C * wl.t * 4          # x, y, dY, x, dX, T, dT
+    if wl.kind == "cached_dw":
+        return 2 * m + wl.C * wl.d * wl.d * e + wl.C * 9 * e   # x, z, M, K
+    return 2 * m + tbl
+
+
+def kernel_bytes(wl, name):
+    e = 2
+    m = wl.B * wl.C * wl.H * wl.W * e
+    tbl = wl.C * wl.t * e
+    return {"forward": 2 * m + tbl, "backward_dx": 2 * m + tbl,
+            "backward_dt": 2 * m + wl.C * wl.t * 4,
+            "forward_cached": 2 * m + wl.C * wl.d * wl.d * e,
+            "dw3x3": 2 * m + wl.C * 9 * e}[name]
+
+
+def kernel_flops(wl, name):
+    n = wl.B * wl.C * wl.H * wl.W
+    if name == "dw3x3":
+        return 18.0 * n
+    return 2.0 * n * wl.d
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during timing."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            out_dir = os.path.join(ROOT, "gpurun_out")
+            os.makedirs(out_dir, exist_ok=True)
+            self.path = os.path.join(out_dir, "clocks_rank%d.csv" % self.gpu)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        sm, smax, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = max(smax, float(parts[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------- GPU arm
+
+class Arm:
+    """Device buffers and the step of one workload (one rank)."""
+
+    def __init__(self, wl, seed, nsets, dev):
+        import windowed_matmul_conv_b200 as wb
+        self.wb = wb
+        self.wl = wl
+        self.dev = dev
+        d = synth.draw(wl, seed=seed)
+        self.host = d
+        self.sets = []
+        for k in range(nsets):
+            s = {"x": d["x"].to(dev)}
+            if k > 0:   # distinct bytes per set so that no set is an L2 copy of another
+                s["x"] = torch.roll(s["x"], shifts=k, dims=0).contiguous()
+            s["y"] = torch.empty_like(s["x"])
+            if wl.kind == "train":
+                s["dY"] = torch.roll(d["dY"].to(dev), shifts=k, dims=0).contiguous()
+                s["dX"] = torch.empty_like(s["x"])
+            self.sets.append(s)
+        self.T = d["T"].to(dev)
+        if wl.kind == "train":
+            self.dT = torch.empty((wl.C, wl.t), dtype=torch.float32, device=dev)
+            nbytes = wb.wbmm_backward_workspace_bytes(wl.B, wl.C, wl.H, wl.W, wl.w, torch.bfloat16)
+            self.ws = torch.empty(max(1, nbytes // 4), dtype=torch.float32, device=dev)
+        if wl.kind == "cached_dw":
+            self.M = wb.cache_matrices(self.T, wl.w)
+            self.K = d["K"].to(dev)
+            for s in self.sets:
+                s["z"] = torch.empty_like(s["x"])
+
+    def kernels(self):
+        k = self.wl.kind
+        if k == "train":
+            return ["forward", "backward_dx", "backward_dt"]
+        if k == "cached_dw":
+            return ["forward_cached", "dw3x3"]
+        return ["forward"]
+
+    def launch(self, name, s):
+        wb, w = self.wb, self.wl.w
+        if name == "forward":
+            wb.wbmm_forward(s["x"], self.T, s["y"], w)
+        elif name == "backward_dx":
+            wb.wbmm_backward(None, self.T, s["dY"], s["dX"], None, None, w)
+        elif name == "backward_dt":
+            wb.wbmm_backward(s["x"], None, s["dY"], None, self.dT, self.ws, w)
+        elif name == "forward_cached":
+            wb.wbmm_forward_cached(s["x"], self.M, None, s["y"], w)
+        elif name == "dw3x3":
+            wb.wbmm_dw3x3(s["y"], self.K, s["z"])
+
+    def step(self, k):
+        s = self.sets[k % len(self.sets)]
+        for name in self.kernels():
+            self.launch(name, s)
+
+
+def barrier(world):
+    if world > 1:
+        dist.barrier()
+
+
+def max_over_ranks(v, world, dev):
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(v, world, dev):
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def prefill(ms=20.0):
+    """Keeps the GPU busy while the host enqueues the timed launches."""
+    torch.cuda._sleep(int(ms * 1e6 * 2.0))   # ~2 GHz cycles per ns
+
+
+def cpu_baseline(wl, host, budget_s=10.0):
+    """The oracle, as it stands, on a bounded sample: the first images of the
+    same inputs (all channels), repeated until `budget_s` of CPU time."""
+    import oracle
+    bs = max(1, min(wl.B, 32 if wl.kind == "train" else 8))
+    sub = wl.scaled(B=bs)
+    x = host["x"][:bs]
+    T = host["T"]
+    runs, t0 = 0, time.perf_counter()
+    while True:
+        if wl.kind == "train":
+            dy = host["dY"][:bs]
+            oracle.forward(x, T, wl.w)
+            oracle.backward_dx(dy, T, wl.w)
+            oracle.backward_dt(x, dy, wl.w)
+        elif wl.kind == "cached_dw":
+            M = oracle.expand(T, wl.w)
+            y = oracle.forward_cached(x, M, wl.w)
+            oracle.dw3x3(y, host["K"])
+        else:
+            oracle.forward(x, T, wl.w)
+        runs += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    tf = step_flops(sub) * runs / el / 1e12
+    return {"value": tf, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": "%d of %d images, all %d channels, %d repetitions, %.1f s (fp64 C loops)"
+                      % (bs, wl.B, wl.C, runs, el)}
+
+
+def run_gpu(args, rank, world, local_rank):
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    wl = synth.WORKLOADS[WORKLOADS[args.workload]]
+    peaks = load_peaks()
+    wb_arm = Arm(wl, seed=rank, nsets=3, dev=dev)
+    wb = wb_arm.wb
+    K, W = args.steps, args.warmup
+    stream = torch.cuda.current_stream()
+
+    # warm-up (also configures kernels before graph capture)
+    for k in range(W):
+        wb_arm.step(k)
+    torch.cuda.synchronize()
+    assert wb.wbmm_get_device_status() == 0, "device status after warm-up"
+
+    # one CUDA graph per buffer set: the step's launches replay back to back
+    graphs = []
+    for k in range(len(wb_arm.sets)):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            wb_arm.step(k)
+        graphs.append(g)
+    for g in graphs:
+        g.replay()
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.3)
+
+    # ---- region A: K steps, device time
+    launches0 = wb.wbmm_launch_count()
+    barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    prefill()
+    e0.record(stream)
+    for k in range(K):
+        graphs[k % len(graphs)].replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms_total = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    ms_step = ms_total / K
+    # graph replays launch the captured kernels: count them per step
+    per_step_launches = len(wb_arm.kernels()) + (1 if wl.kind == "train" else 0)
+    gpu_launches = per_step_launches * K
+    assert wb.wbmm_launch_count() == launches0   # graphs: no host launches
+
+    # ---- region B: the same steps launched eagerly, events around each kernel
+    names = wb_arm.kernels()
+    evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in names] for _ in range(K)]
+    barrier(world)
+    torch.cuda.synchronize()
+    prefill()
+    for k in range(K):
+        s = wb_arm.sets[k % len(wb_arm.sets)]
+        for j, name in enumerate(names):
+            evs[k][j][0].record(stream)
+            wb_arm.launch(name, s)
+            evs[k][j][1].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    kern = {}
+    for j, name in enumerate(names):
+        avg = sum(evs[k][j][0].elapsed_time(evs[k][j][1]) for k in range(K)) / K
+        avg = max_over_ranks(avg, world, dev)
+        gbs = kernel_bytes(wl, name) / (avg * 1e-3) / 1e9
+        kern[name] = {"us": round(avg * 1e3, 2), "gbs": round(gbs, 1),
+                      "tflops": round(kernel_flops(wl, name) / (avg * 1e-3) / 1e12, 2),
+                      "hbm_frac": round(gbs / peaks["hbm_gbs"], 3)}
+    clk = clocks.stop()
+    assert wb.wbmm_get_device_status() == 0, "device status after timing"
+
+    # ---- e2e: pinned host inputs -> device -> step -> host outputs
+    host_in = {"x": wb_arm.host["x"].pin_memory()}
+    if wl.kind == "train":
+        host_in["dY"] = wb_arm.host["dY"].pin_memory()
+    s0 = wb_arm.sets[0]
+    outs = ["y"] if wl.kind == "forward" else (["y", "dX"] if wl.kind == "train" else ["z"])
+    host_out = {o: torch.empty(s0[o].shape, dtype=s0[o].dtype, pin_memory=True) for o in outs}
+    if wl.kind == "train":
+        host_out["dT"] = torch.empty(wb_arm.dT.shape, dtype=torch.float32, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+    ke = max(2, min(K, 10))
+    barrier(world)
+    torch.cuda.synchronize()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for k in range(ke):
+        for nm, t in host_in.items():
+            s0[nm].copy_(t, non_blocking=True)
+        wb_arm.step(0)
+        for nm, t in host_out.items():
+            src = wb_arm.dT if nm == "dT" else s0[nm]
+            t.copy_(src, non_blocking=True)
+    f1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(f0.elapsed_time(f1), world, dev) / ke
+
+    flops_all = sum_over_ranks(step_flops(wl), world, dev)
+    bytes_all = sum_over_ranks(step_bytes(wl), world, dev)
+    value = flops_all / (ms_step * 1e-3) / 1e12
+    result = {
+        "metric": METRIC,
+        "value": round(value, 3),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": W,
+        "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {
+            "workload": "%s: B%d C%d %dx%d w%d (%s)" % (wl.name, wl.B, wl.C, wl.H, wl.W, wl.w,
+                                                      {"train": "forward + dX + dT",
+                                                       "forward": "forward",
+                                                       "cached_dw": "cached forward + 3x3"}[wl.kind]),
+            "B": wl.B, "C_per_gpu": wl.C, "H": wl.H, "W": wl.W, "w": wl.w,
+            "parallelism": "channel-sharded, %d rank(s), no collective" % world,
+            "l2": "3 rotating input/output sets, %.0f MB per step > 126 MB L2"
+                  % (step_bytes(wl) / 1e6),
+            "timing": "CUDA graph replay, CUDA events, max over ranks",
+        },
+        "gbs": round(bytes_all / (ms_step * 1e-3) / 1e9, 1),
+        "windows_channels_per_s": round(sum_over_ranks(wl.windows_per_channel * wl.C, world, dev)
+                                        / (ms_step * 1e-3), 1),
+        "kernels": kern,
+        "gpu_launches": gpu_launches,
+    }
+    # roofline of the dominant kernel (HBM-bound at w <= 14: AI ~ d/2 < ridge)
+    dom = max(kern, key=lambda n: kern[n]["us"])
+    ai = kernel_flops(wl, dom) / kernel_bytes(wl, dom)
+    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    if ai < ridge:
+        result["roofline"] = {"bound": "hbm", "kernel": dom, "achieved": kern[dom]["gbs"],
+                              "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                              "frac": round(kern[dom]["gbs"] / peaks["hbm_gbs"], 4),
+                              "traffic": None, "peak_source": peaks["source"]}
+    else:
+        result["roofline"] = {"bound": "tensor", "kernel": dom, "achieved": kern[dom]["tflops"],
+                              "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                              "frac": round(kern[dom]["tflops"] / peaks["bf16_tflops"], 4),
+                              "traffic": None, "peak_source": peaks["source"]}
+    step_roof_tf = min(peaks["bf16_tflops"], step_flops(wl) / step_bytes(wl) * peaks["hbm_gbs"] / 1e3)
+    result["step_roofline_frac"] = round(value / world / step_roof_tf, 4)
+    result["e2e"] = {"value": round(flops_all / (e2e_ms * 1e-3) / 1e12, 4), "unit": "TFLOP/s",
+                     "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d,
+                     "d2h_bytes_per_step": d2h}
+    if clk is not None:
+        result["clocks"] = clk
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(wl, wb_arm.host)
+    for g in graphs:
+        del g
+    return result
+
+
+def run_reference(args, rank, world):
+    """The oracle as it stands, on host cores, rank 0 only."""
+    if rank != 0:
+        return None
+    import oracle
+    wl = synth.WORKLOADS[WORKLOADS[args.workload]]
+    bs = 8 if wl.kind == "train" else 4
+    sub = wl.scaled(B=min(bs, wl.B))
+    d = synth.draw(wl, seed=0)
+    x, T = d["x"][:sub.B], d["T"]
+
+    def one():
+        if wl.kind == "train":
+            dy = d["dY"][:sub.B]
+            oracle.forward(x, T, wl.w)
+            oracle.backward_dx(dy, T, wl.w)
+            oracle.backward_dt(x, dy, wl.w)
+        elif wl.kind == "cached_dw":
+            y = oracle.forward_cached(x, oracle.expand(T, wl.w), wl.w)
+            oracle.dw3x3(y, d["K"])
+        else:
+            oracle.forward(x, T, wl.w)
+
+    for _ in range(args.warmup):
+        one()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        one()
+    el = time.perf_counter() - t0
+    value = step_flops(sub) * args.steps / el / 1e12
+    sample = "%d of %d images, all %d channels per step (fp64 C loops)" % (sub.B, wl.B, wl.C)
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(el / args.steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "%s: B%d C%d %dx%d w%d, sampled" % (wl.name, wl.B, wl.C, wl.H,
+                                                                   wl.W, wl.w)},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s",
+                         "cores": oracle.num_threads(), "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["wbmm", "reference"], default="wbmm")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="train")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "wbmm":
+        ap.error("at least 3 warm-up steps")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        res = run_gpu(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,277 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle.
+
+Small shapes span several tiles and a ragged last tile for every window size
+class the tensor-core kernels compile (one and two 128-row M tiles, odd and
+even w); the full-size workloads run in the launch configuration the
+benchmark times and are compared on sampled (image, channel) planes, which
+the oracle computes exactly because planes are independent.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from parity_util import (check_bf16, check_f32, dt_bound, forward_rowbound, to_np,
+                         window_norms)
+
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+import windowed_matmul_conv_b200 as wb  # noqa: E402
+
+DEV = "cuda:0"
+
+
+def gen(shape, seed, dtype=torch.bfloat16, scale=1.0):
+    return synth.draw_tensor(shape, seed, "f32", scale).to(dtype).to(DEV)
+
+
+def run_forward(x, T, w):
+    y = wb.forward(x, T, w)
+    torch.cuda.synchronize()
+    assert wb.wbmm_get_device_status() == 0
+    return y
+
+
+# (B, C, H, W, w): several tiles and a ragged tail per shape
+BF16_SHAPES = [
+    (9, 3, 56, 56, 14),     # 36 bands/channel, 16-band tiles -> 16, 16, 4
+    (2, 4, 42, 28, 14),     # nh = 3, nw = 2
+    (5, 2, 105, 112, 7),    # one 128-row M tile, 128-window tiles, ragged
+    (3, 3, 48, 64, 16),     # d = 256, no K padding
+    (4, 2, 39, 104, 13),    # odd w with two M tiles
+    (6, 3, 40, 40, 5),      # odd w, one M tile
+    (3, 2, 24, 48, 3),
+    (2, 2, 24, 96, 12),
+]
+
+
+@pytest.mark.parametrize("shape", BF16_SHAPES, ids=lambda s: "x".join(map(str, s)))
+def test_forward_bf16_small(shape):
+    B, C, H, W, w = shape
+    x = gen((B, C, H, W), 1)
+    T = gen((C, (2 * w - 1) ** 2), 2, scale=0.02)
+    y = run_forward(x, T, w)
+    assert wb.wbmm_last_path() == 1, "tensor-core kernel expected"
+    xr, Tr = to_np(x), to_np(T)
+    ref = oracle.forward(xr, Tr, w)
+    check_bf16(to_np(y), ref, forward_rowbound(xr, Tr, w), "forward")
+
+
+def test_forward_fp32_tiny_workload():
+    wl = synth.WORKLOADS["tiny_fp32"]
+    d = synth.draw(wl, seed=0)
+    x, T = d["x"].to(DEV), d["T"].to(DEV)
+    y = run_forward(x, T, wl.w)
+    ref = oracle.forward(d["x"], d["T"], wl.w)
+    absdot = oracle.forward(np.abs(to_np(d["x"])), np.abs(to_np(d["T"])), wl.w)
+    check_f32(to_np(y), ref, absdot, "tiny fp32 forward")
+
+
+@pytest.mark.parametrize("shape", [(2, 3, 14, 28, 7), (1, 2, 28, 28, 14), (2, 1, 6, 9, 3)])
+def test_fp32_forward_backward(shape):
+    B, C, H, W, w = shape
+    x = gen((B, C, H, W), 3, torch.float32)
+    dy = gen((B, C, H, W), 4, torch.float32)
+    T = gen((C, (2 * w - 1) ** 2), 5, torch.float32, 0.02)
+    xr, gr, Tr = to_np(x), to_np(dy), to_np(T)
+    y = run_forward(x, T, w)
+    check_f32(to_np(y), oracle.forward(xr, Tr, w), oracle.forward(np.abs(xr), np.abs(Tr), w), "y")
+    dX, dT = wb.backward(x, T, dy, w)
+    torch.cuda.synchronize()
+    check_f32(to_np(dX), oracle.backward_dx(gr, Tr, w),
+              oracle.backward_dx(np.abs(gr), np.abs(Tr), w), "dX")
+    absdt = oracle.backward_dt(np.abs(xr), np.abs(gr), w)
+    check_f32(to_np(dT), oracle.backward_dt(xr, gr, w), absdt, "dT")
+
+
+@pytest.mark.parametrize("shape", BF16_SHAPES[:6], ids=lambda s: "x".join(map(str, s)))
+def test_backward_bf16_small(shape):
+    B, C, H, W, w = shape
+    x = gen((B, C, H, W), 6)
+    dy = gen((B, C, H, W), 7)
+    T = gen((C, (2 * w - 1) ** 2), 8, scale=0.02)
+    dX, dT = wb.backward(x, T, dy, w)
+    torch.cuda.synchronize()
+    assert wb.wbmm_get_device_status() == 0
+    assert wb.wbmm_last_path() == 1
+    xr, gr, Tr = to_np(x), to_np(dy), to_np(T)
+    check_bf16(to_np(dX), oracle.backward_dx(gr, Tr, w),
+               forward_rowbound(gr, Tr[:, ::-1].copy(), w), "dX")
+    check_bf16(to_np(dT), oracle.backward_dt(xr, gr, w), dt_bound(xr, gr, w), "dT")
+
+
+def test_dt_is_deterministic():
+    B, C, H, W, w = 9, 3, 56, 56, 14
+    x, dy = gen((B, C, H, W), 9), gen((B, C, H, W), 10)
+    T = gen((C, 729), 11, scale=0.02)
+    runs = []
+    for _ in range(4):
+        _, dT = wb.backward(x, T, dy, w, need_dx=False)
+        runs.append(dT.clone())
+    torch.cuda.synchronize()
+    for r in runs[1:]:
+        assert torch.equal(r, runs[0])
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_cache_matrices_bit_exact(dtype):
+    for w in (3, 7, 14):
+        T = gen((5, (2 * w - 1) ** 2), 12, dtype)
+        M = wb.cache_matrices(T, w)
+        torch.cuda.synchronize()
+        assert np.array_equal(to_np(M), oracle.expand(to_np(T), w))
+
+
+@pytest.mark.parametrize("shape", [(3, 2, 56, 56, 14), (2, 3, 112, 56, 7), (2, 2, 48, 48, 16)])
+def test_forward_cached_bf16(shape):
+    B, C, H, W, w = shape
+    x = gen((B, C, H, W), 13)
+    T = gen((C, (2 * w - 1) ** 2), 14, scale=0.02)
+    M = wb.cache_matrices(T, w)
+    y = wb.forward_cached(x, M, w)
+    torch.cuda.synchronize()
+    assert wb.wbmm_last_path() == 1
+    xr, Tr = to_np(x), to_np(T)
+    check_bf16(to_np(y), oracle.forward(xr, Tr, w), forward_rowbound(xr, Tr, w), "cached")
+    # and the table path gives the identical bits
+    assert torch.equal(y, wb.forward(x, T, w))
+    # any matrix, not only a Toeplitz one
+    Mr = gen((C, w * w, w * w), 15, scale=0.05)
+    y2 = wb.forward_cached(x, Mr, w)
+    torch.cuda.synchronize()
+    Mn = to_np(Mr)
+    ref = oracle.forward_cached(xr, Mn, w)
+    rn = np.sqrt((Mn ** 2).sum(axis=2)).reshape(C, w, w)
+    bound = window_norms(xr, w) * np.tile(rn, (1, H // w, W // w))[None]
+    check_bf16(to_np(y2), ref, bound, "cached random M")
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_dw3x3(dtype):
+    y = gen((3, 4, 37, 70), 16, dtype)
+    K = gen((4, 1, 3, 3), 17, dtype, 1.0 / 3.0)
+    z = wb.dw3x3(y, K)
+    torch.cuda.synchronize()
+    yr, Kr = to_np(y), to_np(K)
+    ref = oracle.dw3x3(yr, Kr)
+    if dtype == torch.float32:
+        absdot = oracle.dw3x3(np.abs(yr), np.abs(Kr))
+        check_f32(to_np(z), ref, absdot, "dw3x3 fp32")
+    else:
+        bound = oracle.dw3x3(np.abs(yr), np.abs(Kr))
+        check_bf16(to_np(z), ref, bound, "dw3x3 bf16")
+
+
+def test_guard_bands_untouched():
+    B, C, H, W, w = 9, 3, 56, 56, 14
+    n = B * C * H * W
+    pad = 4096
+    x = gen((B, C, H, W), 18)
+    T = gen((C, 729), 19, scale=0.02)
+    buf = torch.full((n + 2 * pad,), 7.0, dtype=torch.bfloat16, device=DEV)
+    y = buf[pad:pad + n].view(B, C, H, W)
+    wb.wbmm_forward(x, T, y, w)
+    torch.cuda.synchronize()
+    assert torch.all(buf[:pad] == 7.0) and torch.all(buf[pad + n:] == 7.0)
+    assert torch.equal(y, wb.forward(x, T, w))
+
+
+def test_argument_errors_launch_nothing():
+    x = gen((1, 2, 28, 28), 20)
+    T = gen((2, 729), 21, scale=0.02)
+    y = torch.empty_like(x)
+    before = wb.wbmm_launch_count()
+    with pytest.raises(wb.WbmmError) as e:
+        wb.wbmm_forward(x, T, y, 5)                    # 28 % 5 != 0
+    assert e.value.status == 2
+    with pytest.raises(wb.WbmmError) as e:
+        wb.wbmm_forward(x, T, x, 14)                   # output overlaps input
+    assert e.value.status == 1
+    big = torch.empty(x.numel() + 8, dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(wb.WbmmError) as e:
+        wb.wbmm_forward(x, T, big[1:1 + x.numel()].view_as(x), 14)  # 2-byte offset
+    assert e.value.status == 4
+    dT = torch.empty((2, 729), dtype=torch.float32, device=DEV)
+    ws = torch.empty(4, dtype=torch.float32, device=DEV)
+    with pytest.raises(wb.WbmmError) as e:
+        wb.wbmm_backward(x, T, x, None, dT, ws, 14)    # workspace too small
+    assert e.value.status == 6
+    assert wb.wbmm_launch_count() == before
+
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    wb.wbmm_wait_selftest(2_000_000)
+    assert wb.wbmm_get_device_status() == 8
+    assert wb.wbmm_get_device_status() == 0          # cleared
+    x = gen((2, 2, 28, 28), 22)
+    T = gen((2, 729), 23, scale=0.02)
+    y = run_forward(x, T, 14)
+    ref = oracle.forward(to_np(x), to_np(T), 14)
+    check_bf16(to_np(y), ref, forward_rowbound(to_np(x), to_np(T), 14), "after timeout")
+
+
+# ---------------------------------------------------------------- full size
+
+def sample_planes(B, C, nb=3, nc=3, seed=0):
+    g = np.random.default_rng(seed)
+    bs = sorted(set([0, B - 1] + list(g.integers(0, B, nb))))
+    cs = sorted(set([0, C - 1] + list(g.integers(0, C, nc))))
+    return bs, cs
+
+
+@pytest.mark.parametrize("name", ["fwd_bf16", "sweep_w7", "sweep_w14", "sweep_w28"])
+def test_full_size_forward_sampled(name):
+    wl = synth.WORKLOADS[name]
+    d = synth.draw(wl, seed=0)
+    x, T = d["x"].to(DEV), d["T"].to(DEV)
+    y = run_forward(x, T, wl.w)
+    bs, cs = sample_planes(wl.B, wl.C)
+    xs = to_np(d["x"][bs][:, cs])
+    Ts = to_np(d["T"][cs])
+    ref = oracle.forward(xs, Ts, wl.w)
+    got = to_np(y[bs][:, cs])
+    check_bf16(got, ref, forward_rowbound(xs, Ts, wl.w), name)
+
+
+def test_full_size_training_step_sampled():
+    wl = synth.WORKLOADS["train_bf16"]
+    d = synth.draw(wl, seed=0)
+    x, T, dy = d["x"].to(DEV), d["T"].to(DEV), d["dY"].to(DEV)
+    y = run_forward(x, T, wl.w)
+    dX, dT = wb.backward(x, T, dy, wl.w)
+    torch.cuda.synchronize()
+    assert wb.wbmm_get_device_status() == 0
+    bs, cs = sample_planes(wl.B, wl.C)
+    xs, gs, Ts = to_np(d["x"][bs][:, cs]), to_np(d["dY"][bs][:, cs]), to_np(d["T"][cs])
+    check_bf16(to_np(y[bs][:, cs]), oracle.forward(xs, Ts, wl.w),
+               forward_rowbound(xs, Ts, wl.w), "train y")
+    check_bf16(to_np(dX[bs][:, cs]), oracle.backward_dx(gs, Ts, wl.w),
+               forward_rowbound(gs, Ts[:, ::-1].copy(), wl.w), "train dX")
+    # dT of a channel sums over every image: the oracle takes whole channels
+    xc, gc = to_np(d["x"][:, cs]), to_np(d["dY"][:, cs])
+    check_bf16(to_np(dT[cs]), oracle.backward_dt(xc, gc, wl.w), dt_bound(xc, gc, wl.w),
+               "train dT")
+
+
+def test_full_size_cached_dw_sampled():
+    wl = synth.WORKLOADS["hires_cached_dw"]
+    d = synth.draw(wl, seed=0)
+    x, T, K = d["x"].to(DEV), d["T"].to(DEV), d["K"].to(DEV)
+    M = wb.cache_matrices(T, wl.w)
+    y = wb.forward_cached(x, M, wl.w)
+    z = wb.dw3x3(y, K)
+    torch.cuda.synchronize()
+    assert wb.wbmm_get_device_status() == 0
+    bs, cs = sample_planes(wl.B, wl.C)
+    xs, Ts, Ks = to_np(d["x"][bs][:, cs]), to_np(d["T"][cs]), to_np(d["K"][cs])
+    yref = oracle.forward(xs, Ts, wl.w)
+    check_bf16(to_np(y[bs][:, cs]), yref, forward_rowbound(xs, Ts, wl.w), "hires y")
+    zref = oracle.dw3x3(yref, Ks)
+    # |z - zref| <= sum |K| * (|y - yref| + rounding of z): bound by the 3x3 of
+    # the forward row bound
+    zb = oracle.dw3x3(forward_rowbound(xs, Ts, wl.w), np.abs(Ks))
+    check_bf16(to_np(z[bs][:, cs]), zref, zb, "hires z")

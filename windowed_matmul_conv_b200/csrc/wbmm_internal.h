@@ -1,0 +1,71 @@
+// Host-side interface between the C ABI layer and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+namespace wbmm {
+
+// Geometry of one call.  Bands are the w-row strips of one image plane: band
+// g = b*nh + i of channel c holds windows (b, i, 0..nw-1) and is w*W
+// contiguous elements of the NCHW map.
+struct Geom {
+    int B, C, H, W, w;
+    int nh, nw, d, tsz;
+    long long bands;     // B * nh bands per channel
+};
+
+inline Geom make_geom(int B, int C, int H, int W, int w)
+{
+    Geom g;
+    g.B = B; g.C = C; g.H = H; g.W = W; g.w = w;
+    g.nh = H / w; g.nw = W / w; g.d = w * w; g.tsz = (2 * w - 1) * (2 * w - 1);
+    g.bands = (long long)B * g.nh;
+    return g;
+}
+
+// How the tensor-core kernel builds its A operand (the per-channel matrix).
+enum AMode : int {
+    kTable = 0,      // M_c[u][v] from the table (forward)
+    kTableFlip = 1,  // M_c[v][u] from the table (input gradient)
+    kCached = 2,     // M_c read from a [C][d][d] matrix in global memory
+};
+
+struct Launch {
+    cudaStream_t stream;
+    int num_sms;
+    int* status;                  // device status word
+    unsigned long long budget;    // bounded-wait budget, SM cycles
+};
+
+// tcgen05 forward family (x: bf16 map; src: table or matrices; dw: fused 3x3
+// weights or null).  *_supported() must be checked before launching.
+bool tc_fwd_supported(const Geom& g, bool fused);
+cudaError_t tc_fwd_launch(const Geom& g, AMode mode, const void* x, const void* src, void* y,
+                          const void* dw, const Launch& L);
+
+// tcgen05 table gradient: per (channel, chunk) fp32 partial tables.
+bool tc_dt_supported(const Geom& g);
+int tc_dt_chunks(const Geom& g);
+cudaError_t tc_dt_launch(const Geom& g, const void* x, const void* dy, float* partials,
+                         const Launch& L);
+
+// CUDA-core kernels.  is_bf16 selects the element type of every map/table.
+int simt_dt_chunks(const Geom& g);
+cudaError_t simt_fwd_launch(const Geom& g, AMode mode, bool is_bf16, const void* x,
+                            const void* src, void* y, const Launch& L);
+cudaError_t simt_dt_launch(const Geom& g, bool is_bf16, const void* x, const void* dy,
+                           float* partials, const Launch& L);
+cudaError_t dt_finalize_launch(int C, int tsz, int chunks, const float* partials, float* dT,
+                               const Launch& L);
+cudaError_t cache_matrices_launch(int C, int w, bool is_bf16, const void* T, void* M,
+                                  const Launch& L);
+cudaError_t dw3x3_launch(const Geom& g, bool is_bf16, const void* y, const void* K, void* z,
+                         const Launch& L);
+cudaError_t wait_selftest_launch(unsigned long long cycles, const Launch& L);
+
+void note_launches(int n);
+
+}  // namespace wbmm

@@ -1,0 +1,356 @@
+// CUDA-core kernels: the fp32 WBMM path (tensor-core tf32 cannot meet the
+// fp32 accuracy bound), bf16 shapes outside the tensor-core kernels' limits,
+// the table-gradient finaliser, matrix caching, the standalone 3x3 depthwise
+// mixing and the bounded-wait self-test.
+#include <cuda_bf16.h>
+
+#include "ptx_sm100.cuh"
+#include "wbmm_internal.h"
+
+namespace wbmm {
+
+__device__ __forceinline__ float to_f(float v) { return v; }
+__device__ __forceinline__ float to_f(__nv_bfloat16 v) { return __bfloat162float(v); }
+template <typename T>
+__device__ __forceinline__ T from_f(float v);
+template <>
+__device__ __forceinline__ float from_f<float>(float v) { return v; }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float v)
+{
+    return __float2bfloat16_rn(v);
+}
+
+// ------------------------------------------------------------- forward
+// One block per band (plane b*C+c, window row i): the band's w rows and the
+// channel's table sit in shared memory as fp32; each thread computes outputs
+// (window j, position u) with an fp32 sum in fixed (r, s) order.
+template <typename TIn>
+__global__ void simt_fwd_kernel(const TIn* __restrict__ x, const TIn* __restrict__ src,
+                                TIn* __restrict__ y, int C, int H, int W, int w, int nh, int nw,
+                                int mode)
+{
+    extern __shared__ float sm[];
+    const int tsz = (2 * w - 1) * (2 * w - 1), d = w * w;
+    const long long blk = blockIdx.x;
+    const long long bc = blk / nh;
+    const int i = (int)(blk - bc * nh);
+    const int c = (int)(bc % C);
+    float* tbl = sm;
+    float* band = sm + (mode == kCached ? 0 : tsz);
+    if (mode != kCached)
+        for (int k = threadIdx.x; k < tsz; k += blockDim.x)
+            tbl[k] = to_f(src[(long long)c * tsz + k]);
+    const TIn* xb = x + (bc * H + (long long)i * w) * W;
+    for (int k = threadIdx.x; k < w * W; k += blockDim.x)
+        band[k] = to_f(xb[k]);
+    __syncthreads();
+    TIn* yb = y + (bc * H + (long long)i * w) * W;
+    const TIn* Mc = src + (long long)c * d * d;
+    for (int o = threadIdx.x; o < nw * d; o += blockDim.x) {
+        const int j = o / d, u = o - (o / d) * d;
+        const int p = u / w, q = u - (u / w) * w;
+        float acc = 0.0f;
+        for (int r = 0; r < w; ++r) {
+            const float* xr = band + r * W + j * w;
+            const int rowi = (p - r + w - 1) * (2 * w - 1) + (q + w - 1);
+            for (int s = 0; s < w; ++s) {
+                float coef;
+                if (mode == kCached)
+                    coef = to_f(Mc[(long long)u * d + r * w + s]);
+                else if (mode == kTableFlip)
+                    coef = tbl[tsz - 1 - (rowi - s)];
+                else
+                    coef = tbl[rowi - s];
+                acc = __fmaf_rn(coef, xr[s], acc);
+            }
+        }
+        yb[p * W + j * w + q] = from_f<TIn>(acc);
+    }
+}
+
+// ------------------------------------------------------- table gradient
+// One block per (channel, chunk of kSimtChunkBands bands); each thread owns
+// table bins and sums dy[p,q] * x[p-dp, q-dq] over the chunk's windows in a
+// fixed order.  Partials go to [C][chunks][tsz].
+constexpr int kSimtChunkBands = 8;
+constexpr int kSimtMaxBinsPerThread = 16;
+
+template <typename TIn>
+__global__ void simt_dt_kernel(const TIn* __restrict__ x, const TIn* __restrict__ dy,
+                               float* __restrict__ part, int C, int H, int W, int w, int nh,
+                               int nw, long long bands, int chunks)
+{
+    extern __shared__ float sm[];
+    const int tsz = (2 * w - 1) * (2 * w - 1);
+    const int c = blockIdx.x / chunks, k = blockIdx.x - (blockIdx.x / chunks) * chunks;
+    float* xb = sm;
+    float* gb = sm + w * W;
+    float acc[kSimtMaxBinsPerThread];
+    for (int m = 0; m < kSimtMaxBinsPerThread; ++m)
+        acc[m] = 0.0f;
+    const long long g0 = (long long)k * kSimtChunkBands;
+    const long long g1 = g0 + kSimtChunkBands < bands ? g0 + kSimtChunkBands : bands;
+    for (long long g = g0; g < g1; ++g) {
+        const long long b = g / nh;
+        const int i = (int)(g - b * nh);
+        const long long off = ((b * C + c) * H + (long long)i * w) * W;
+        __syncthreads();
+        for (int e = threadIdx.x; e < w * W; e += blockDim.x) {
+            xb[e] = to_f(x[off + e]);
+            gb[e] = to_f(dy[off + e]);
+        }
+        __syncthreads();
+        for (int m = 0; m < kSimtMaxBinsPerThread; ++m) {
+            const int t = threadIdx.x + m * blockDim.x;
+            if (t >= tsz)
+                break;
+            const int dp = t / (2 * w - 1) - (w - 1), dq = t % (2 * w - 1) - (w - 1);
+            const int p0 = dp > 0 ? dp : 0, p1 = dp > 0 ? w : w + dp;
+            const int q0 = dq > 0 ? dq : 0, q1 = dq > 0 ? w : w + dq;
+            float a = acc[m];
+            for (int j = 0; j < nw; ++j)
+                for (int p = p0; p < p1; ++p)
+                    for (int q = q0; q < q1; ++q)
+                        a = __fmaf_rn(gb[p * W + j * w + q], xb[(p - dp) * W + j * w + (q - dq)],
+                                      a);
+            acc[m] = a;
+        }
+    }
+    for (int m = 0; m < kSimtMaxBinsPerThread; ++m) {
+        const int t = threadIdx.x + m * blockDim.x;
+        if (t < tsz)
+            part[((long long)c * chunks + k) * tsz + t] = acc[m];
+    }
+}
+
+// Fixed-order sum of the partial tables.
+__global__ void dt_finalize_kernel(const float* __restrict__ part, float* __restrict__ dT, int C,
+                                   int tsz, int chunks)
+{
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= (long long)C * tsz)
+        return;
+    const long long c = i / tsz, t = i - (i / tsz) * tsz;
+    float acc = 0.0f;
+    for (int k = 0; k < chunks; ++k)
+        acc += part[(c * chunks + k) * tsz + t];
+    dT[i] = acc;
+}
+
+// M[c][u][v] = T[c][idx(u, v)]: a bit copy of table entries.
+template <typename E>
+__global__ void cache_kernel(const E* __restrict__ T, E* __restrict__ M, int C, int w)
+{
+    const int d = w * w, tsz = (2 * w - 1) * (2 * w - 1);
+    const long long total = (long long)C * d * d;
+    for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < total;
+         e += (long long)gridDim.x * blockDim.x) {
+        const long long c = e / ((long long)d * d);
+        const int rem = (int)(e - c * d * d);
+        const int u = rem / d, v = rem - (rem / d) * d;
+        const int p = u / w, q = u - (u / w) * w, r = v / w, s = v - (v / w) * w;
+        M[e] = T[c * tsz + (p - r + w - 1) * (2 * w - 1) + (q - s + w - 1)];
+    }
+}
+
+// --------------------------------------------------------- 3x3 mixing
+// Tile of kDwTH x kDwTW outputs with a one-pixel halo (zero outside the
+// image) in shared memory; fp32 sum in fixed (a, e) order.
+constexpr int kDwTH = 16, kDwTW = 64;
+
+template <typename TIn>
+__global__ void dw3x3_kernel(const TIn* __restrict__ y, const TIn* __restrict__ K,
+                             TIn* __restrict__ z, int C, int H, int W, int tiles_y, int tiles_x)
+{
+    __shared__ float tile[(kDwTH + 2) * (kDwTW + 2)];
+    const long long blk = blockIdx.x;
+    const long long bc = blk / ((long long)tiles_y * tiles_x);
+    const int rem = (int)(blk - bc * tiles_y * tiles_x);
+    const int ty = rem / tiles_x, tx = rem - (rem / tiles_x) * tiles_x;
+    const int c = (int)(bc % C);
+    float k[9];
+#pragma unroll
+    for (int m = 0; m < 9; ++m)
+        k[m] = to_f(K[c * 9 + m]);
+    const int h0 = ty * kDwTH, x0 = tx * kDwTW;
+    const TIn* yp = y + bc * H * (long long)W;
+    for (int e = threadIdx.x; e < (kDwTH + 2) * (kDwTW + 2); e += blockDim.x) {
+        const int hh = h0 - 1 + e / (kDwTW + 2), xx = x0 - 1 + e % (kDwTW + 2);
+        tile[e] = (hh >= 0 && hh < H && xx >= 0 && xx < W) ? to_f(yp[(long long)hh * W + xx])
+                                                            : 0.0f;
+    }
+    __syncthreads();
+    TIn* zp = z + bc * H * (long long)W;
+    for (int o = threadIdx.x; o < kDwTH * kDwTW; o += blockDim.x) {
+        const int oh = o / kDwTW, ox = o - (o / kDwTW) * kDwTW;
+        const int h = h0 + oh, xw = x0 + ox;
+        if (h >= H || xw >= W)
+            continue;
+        float acc = 0.0f;
+#pragma unroll
+        for (int a = 0; a < 3; ++a)
+#pragma unroll
+            for (int e = 0; e < 3; ++e)
+                acc = __fmaf_rn(k[a * 3 + e], tile[(oh + a) * (kDwTW + 2) + ox + e], acc);
+        zp[(long long)h * W + xw] = from_f<TIn>(acc);
+    }
+}
+
+// ------------------------------------------------ bounded-wait self-test
+__global__ void wait_selftest_kernel(unsigned long long cycles, int* status)
+{
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    // Nothing ever arrives on `bar`: the wait must give up after `cycles`.
+    if (threadIdx.x == 0)
+        mbar_wait(&bar, 0, &abort_flag, cycles, status);
+}
+
+// ------------------------------------------------------------------ host
+namespace {
+
+template <typename K>
+cudaError_t set_smem(K kernel, size_t bytes)
+{
+    if (bytes <= 48 * 1024)
+        return cudaSuccess;
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+constexpr size_t kSimtSmemMax = 200 * 1024;
+
+}  // namespace
+
+int simt_dt_chunks(const Geom& g)
+{
+    return (int)((g.bands + kSimtChunkBands - 1) / kSimtChunkBands);
+}
+
+cudaError_t simt_fwd_launch(const Geom& g, AMode mode, bool is_bf16, const void* x,
+                            const void* src, void* y, const Launch& L)
+{
+    const size_t smem = ((mode == kCached ? 0 : (size_t)g.tsz) + (size_t)g.w * g.W) * 4;
+    if (smem > kSimtSmemMax)
+        return cudaErrorInvalidConfiguration;
+    const long long blocks = (long long)g.B * g.C * g.nh;
+    if (blocks == 0)
+        return cudaSuccess;
+    if (blocks > 0x7fffffffLL)
+        return cudaErrorInvalidConfiguration;
+    cudaError_t e;
+    if (is_bf16) {
+        e = set_smem(simt_fwd_kernel<__nv_bfloat16>, smem);
+        if (e != cudaSuccess)
+            return e;
+        simt_fwd_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, smem, L.stream>>>(
+            static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(src),
+            static_cast<__nv_bfloat16*>(y), g.C, g.H, g.W, g.w, g.nh, g.nw, (int)mode);
+    } else {
+        e = set_smem(simt_fwd_kernel<float>, smem);
+        if (e != cudaSuccess)
+            return e;
+        simt_fwd_kernel<float><<<(unsigned)blocks, 256, smem, L.stream>>>(
+            static_cast<const float*>(x), static_cast<const float*>(src), static_cast<float*>(y),
+            g.C, g.H, g.W, g.w, g.nh, g.nw, (int)mode);
+    }
+    note_launches(1);
+    return cudaGetLastError();
+}
+
+cudaError_t simt_dt_launch(const Geom& g, bool is_bf16, const void* x, const void* dy,
+                           float* partials, const Launch& L)
+{
+    const size_t smem = (size_t)2 * g.w * g.W * 4;
+    if (smem > kSimtSmemMax || g.tsz > 256 * kSimtMaxBinsPerThread)
+        return cudaErrorInvalidConfiguration;
+    const int chunks = simt_dt_chunks(g);
+    const long long blocks = (long long)g.C * chunks;
+    if (blocks == 0)
+        return cudaSuccess;
+    cudaError_t e;
+    if (is_bf16) {
+        e = set_smem(simt_dt_kernel<__nv_bfloat16>, smem);
+        if (e != cudaSuccess)
+            return e;
+        simt_dt_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, smem, L.stream>>>(
+            static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(dy),
+            partials, g.C, g.H, g.W, g.w, g.nh, g.nw, g.bands, chunks);
+    } else {
+        e = set_smem(simt_dt_kernel<float>, smem);
+        if (e != cudaSuccess)
+            return e;
+        simt_dt_kernel<float><<<(unsigned)blocks, 256, smem, L.stream>>>(
+            static_cast<const float*>(x), static_cast<const float*>(dy), partials, g.C, g.H, g.W,
+            g.w, g.nh, g.nw, g.bands, chunks);
+    }
+    note_launches(1);
+    return cudaGetLastError();
+}
+
+cudaError_t dt_finalize_launch(int C, int tsz, int chunks, const float* partials, float* dT,
+                               const Launch& L)
+{
+    const long long n = (long long)C * tsz;
+    if (n == 0)
+        return cudaSuccess;
+    dt_finalize_kernel<<<(unsigned)((n + 255) / 256), 256, 0, L.stream>>>(partials, dT, C, tsz,
+                                                                         chunks);
+    note_launches(1);
+    return cudaGetLastError();
+}
+
+cudaError_t cache_matrices_launch(int C, int w, bool is_bf16, const void* T, void* M,
+                                  const Launch& L)
+{
+    const long long total = (long long)C * w * w * w * w;
+    long long blocks = (total + 255) / 256;
+    if (blocks > (long long)L.num_sms * 32)
+        blocks = (long long)L.num_sms * 32;
+    if (blocks < 1)
+        return cudaSuccess;
+    if (is_bf16)
+        cache_kernel<uint16_t><<<(unsigned)blocks, 256, 0, L.stream>>>(
+            static_cast<const uint16_t*>(T), static_cast<uint16_t*>(M), C, w);
+    else
+        cache_kernel<uint32_t><<<(unsigned)blocks, 256, 0, L.stream>>>(
+            static_cast<const uint32_t*>(T), static_cast<uint32_t*>(M), C, w);
+    note_launches(1);
+    return cudaGetLastError();
+}
+
+cudaError_t dw3x3_launch(const Geom& g, bool is_bf16, const void* y, const void* K, void* z,
+                         const Launch& L)
+{
+    const int ty = (g.H + kDwTH - 1) / kDwTH, tx = (g.W + kDwTW - 1) / kDwTW;
+    const long long blocks = (long long)g.B * g.C * ty * tx;
+    if (blocks == 0)
+        return cudaSuccess;
+    if (blocks > 0x7fffffffLL)
+        return cudaErrorInvalidConfiguration;
+    if (is_bf16)
+        dw3x3_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, L.stream>>>(
+            static_cast<const __nv_bfloat16*>(y), static_cast<const __nv_bfloat16*>(K),
+            static_cast<__nv_bfloat16*>(z), g.C, g.H, g.W, ty, tx);
+    else
+        dw3x3_kernel<float><<<(unsigned)blocks, 256, 0, L.stream>>>(
+            static_cast<const float*>(y), static_cast<const float*>(K), static_cast<float*>(z),
+            g.C, g.H, g.W, ty, tx);
+    note_launches(1);
+    return cudaGetLastError();
+}
+
+cudaError_t wait_selftest_launch(unsigned long long cycles, const Launch& L)
+{
+    wait_selftest_kernel<<<1, 32, 0, L.stream>>>(cycles, L.status);
+    note_launches(1);
+    return cudaGetLastError();
+}
+
+}  // namespace wbmm
