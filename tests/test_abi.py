@@ -64,8 +64,12 @@ def test_workspace_size_formula(lib):
     f.restype = ctypes.c_size_t
     f.argtypes = [ctypes.c_int] * 6
     # training workload: 64-window tiles of 32 two-window bands, 8 tiles per
-    # channel, chunks of 2 tiles -> 4 fp32 partial tables per channel
-    assert f(128, 256, 28, 28, 14, 1) == 256 * 4 * 729 * 4
+    # channel, one chunk of up to 16 tiles -> 1 fp32 partial table per channel
+    assert f(128, 256, 28, 28, 14, 1) == 256 * 1 * 729 * 4
+    # 64 images of 56x56: 16 bands/tile, 16 tiles/channel -> 1 chunk
+    assert f(64, 128, 56, 56, 14, 1) == 128 * 1 * 729 * 4
+    # 32 images of 112x112: 8 bands/tile, 32 tiles/channel -> 2 chunks
+    assert f(32, 4, 112, 112, 14, 1) == 4 * 2 * 729 * 4
     assert f(1, 1, 14, 15, 7, 1) == 0
 
 

@@ -40,6 +40,17 @@ struct Launch {
     unsigned long long budget;    // bounded-wait budget, SM cycles
 };
 
+// Opaque storage for a CUtensorMap (128 bytes, 64-byte aligned), so kernel
+// parameter structs can hold one without including the driver header.
+struct alignas(64) TmapBytes {
+    unsigned char b[128];
+};
+
+// Tensor maps (see wbmm_tmap.cu).  `map` points at a 64-byte aligned
+// 128-byte CUtensorMap.  Returns false when the shape cannot use one.
+int plane_row_elems(const Geom& g);
+bool encode_plane_map(void* map, const void* base, const Geom& g, int k_images);
+
 // tcgen05 forward family (x: bf16 map; src: table or matrices; dw: fused 3x3
 // weights or null).  *_supported() must be checked before launching.
 bool tc_fwd_supported(const Geom& g, bool fused);

@@ -1,6 +1,7 @@
 // Tensor-core (tcgen05) WBMM table gradient.
 //
-// For one channel, G = dY X^T is a d x d matrix summed over windows:
+// For one channel, G = dY X^T is a matrix over in-window positions summed
+// over windows:
 //   G[u, v] = sum_n dY[u, n] X[v, n]        (u, v in-window positions)
 // and the table gradient is its sum along constant relative offset:
 //   dT[(p-r+w-1)(2w-1) + (q-s+w-1)] = sum over (u=(p,q), v=(r,s)) of G[u, v].
@@ -10,47 +11,63 @@
 // fp32 partial table, so the result is bit-identical from run to run and for
 // any grid size; a second kernel adds the partials in chunk order.
 //
-// Per tile (64 windows = the MMA's K for this GEMM) the producer bulk-copies
-// the dY and x bands into a raw slot; the transform warps write both as
-// K-major operands (rows = positions, K = windows); one thread issues
-// 128 x NP x 16 MMAs into G held in TMEM (two 128-row halves for d > 128).
-// After the item's last tile the epilogue warps read G from TMEM and add each
-// entry into a per-warp bin array in shared memory (within one TMEM column
-// every lane maps to a different bin, so the adds never collide), then sum the
+// Per tile the producer bulk-copies the dY and x bands into a raw slot; the
+// transform warps write both tiles in the layout of the forward kernel's
+// operand (rows = windows, 16-byte rows of 8 padded positions); warps 2..9 do this.  Read as an
+// MN-major operand that layout has positions as M (or N) and windows as K,
+// so one thread issues 128 x NPOS x 16 MMAs (A = dY tile, B = x tile) into G
+// in TMEM (two 128-row halves when the padded positions exceed 128).  After
+// the item's last tile the epilogue warps read G from TMEM and add each entry
+// into a per-warp bin array in shared memory (within one TMEM column every
+// lane maps to a different bin, so the adds never collide), then sum the
 // four warp arrays in warp order into the item's partial table.
 #include <cuda_bf16.h>
 
 #include "ptx_sm100.cuh"
+#include "tc_common.cuh"
 #include "wbmm_internal.h"
 
 namespace wbmm {
 
+constexpr uint32_t kSmemMax = 232448;
+constexpr int kDtRing = 2;
+constexpr int kDtXformWarps = 8;                 // warps 2..9
+constexpr int kDtEpiWarp0 = 2 + kDtXformWarps;  // warps 10..13
+constexpr int kDtThreads = (kDtEpiWarp0 + 4) * 32;
+
+// Shared memory of the dT kernel for window size ws and nt windows per tile:
+// two operand stages (dY and x tiles), the raw ring, per-warp bins, barriers.
+constexpr uint32_t dt_smem_bytes(int ws, int nt)
+{
+    const int d = ws * ws, rp = (ws + 7) / 8 * 8, kp = (ws * rp + 15) / 16 * 16;
+    const uint32_t stage = 2u * (uint32_t)nt * kp * 2;
+    const uint32_t raw = 2u * (uint32_t)((nt * d * 2 + 127) / 128 * 128);
+    const uint32_t bins = 4u * (2 * ws - 1) * (2 * ws - 1) * 4;
+    return 2 * stage + kDtRing * raw + bins + nt * 4 + 2048;
+}
+
+// Windows per tile: 64 when the layout fits, else 32 (w >= 15).
+constexpr int dt_nt_for(int ws) { return dt_smem_bytes(ws, 64) <= kSmemMax ? 64 : 32; }
+
 template <int WS>
-struct DtCfg {
-    static constexpr int D = WS * WS;
-    static constexpr int MT = (D + 127) / 128;
-    static constexpr int NP = (D + 15) / 16 * 16;           // MMA N (positions of x)
-    static constexpr int NT = 64;                           // windows per tile = K per stage
-    static constexpr int KSTEPS = NT / 16;
-    static constexpr int TSZ = (2 * WS - 1) * (2 * WS - 1);
-    static constexpr uint32_t SBO = NT * 16;                // bytes per 8-row group
-    static constexpr int RG = (D + 7) / 8;                  // written 8-row groups
-    // Rows of the A tile past D are never stored; the MMA may read them from
-    // the B tile that follows (their products land in ignored rows of G).
-    static constexpr int A_GROUPS = ((MT * 128 - RG * 8) <= NP) ? RG : MT * 16;
-    static constexpr uint32_t A_BYTES = A_GROUPS * SBO;
-    static constexpr uint32_t B_BYTES = (NP / 8) * SBO;
-    static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
-    static constexpr uint32_t RAW_HALF = (uint32_t)((NT * D * 2 + 127) / 128 * 128);
-    static constexpr uint32_t RAW_BYTES = 2 * RAW_HALF;    // dY tile, then x tile
-    static constexpr uint32_t IDESC = idesc_bf16(128, NP);
-    static_assert(MT * 256 <= 512 || MT == 1, "G must fit in TMEM");
+struct DtCfg : PadCfg<WS> {
+    using P = PadCfg<WS>;
+    static constexpr int NT = dt_nt_for(WS);               // windows per tile = K per stage
+    static constexpr int MT = (P::K + 127) / 128;           // 128-row halves of G
+    static constexpr int NPOS = P::KP;                      // MMA N: padded positions of x
+    static constexpr uint32_t SBO_T = (uint32_t)(P::KP * 16);   // 8-window group stride
+    static constexpr uint32_t TILE_BYTES = (uint32_t)(NT * P::KP * 2);
+    static constexpr uint32_t STAGE_BYTES = 2 * TILE_BYTES;     // dY tile, then x tile
+    static constexpr uint32_t RAW_HALF = (uint32_t)((NT * P::D * 2 + 127) / 128 * 128);
+    static constexpr uint32_t RAW_BYTES = 2 * RAW_HALF;
+    // kind::f16, bf16 A and B, both MN-major (positions contiguous), fp32 D
+    static constexpr uint32_t IDESC = idesc_bf16(128, NPOS) | (1u << 15) | (1u << 16);
+    static_assert(NPOS <= 256 && MT <= 2, "G must fit in TMEM");
 };
 
-constexpr int kDtThreads = 320;
-constexpr int kDtRing = 2;
-
 struct TcDtParams {
+    TmapBytes map_x;        // whole-plane tensor maps (used when use_tmap)
+    TmapBytes map_dy;
     const uint16_t* x;
     const uint16_t* dy;
     float* partials;        // [C][chunks][tsz]
@@ -59,8 +76,10 @@ struct TcDtParams {
     int tpc;                // tiles per channel
     int ch;                 // tiles per chunk
     int chunks;             // chunks per channel
-    long long bands;
-    long long items;        // C * chunks
+    int bands;
+    int items;              // C * chunks
+    int use_tmap;           // tiles are whole planes: one 4-D TMA per tensor
+    int kimg;               // planes per tile when use_tmap
     uint32_t off_raw, off_stage, off_bins, off_woff, off_bar;
     unsigned long long budget;
     int* status;
@@ -79,18 +98,16 @@ struct DtBars {
 };
 
 struct DtTile {
-    int c;
-    long long band0;
-    int nb;
+    BandTile bt;
     bool first, last;   // first / last tile of its item
 };
 
 // The flattened tile sequence of a CTA: items blockIdx.x, +grid, ...; within
 // an item its tiles in order.  Every role walks the same sequence.
 struct DtWalker {
-    long long item;
+    int item;
     int tile;       // tile index within the channel
-    int tile_end;
+    int tile0, tile_end;
     __device__ __forceinline__ bool valid(const TcDtParams& P) const { return item < P.items; }
     __device__ __forceinline__ void start(const TcDtParams& P)
     {
@@ -101,19 +118,18 @@ struct DtWalker {
     {
         if (item >= P.items)
             return;
-        const int chunk = (int)(item % P.chunks);
-        tile = chunk * P.ch;
-        tile_end = tile + P.ch < P.tpc ? tile + P.ch : P.tpc;
+        tile0 = (item % P.chunks) * P.ch;
+        tile = tile0;
+        tile_end = tile0 + P.ch < P.tpc ? tile0 + P.ch : P.tpc;
     }
     __device__ __forceinline__ DtTile get(const TcDtParams& P) const
     {
         DtTile t;
-        t.c = (int)(item / P.chunks);
-        t.band0 = (long long)tile * P.bpt;
-        const long long left = P.bands - t.band0;
-        t.nb = (int)(left < P.bpt ? left : P.bpt);
-        const int chunk = (int)(item % P.chunks);
-        t.first = tile == chunk * P.ch;
+        t.bt.c = item / P.chunks;
+        t.bt.band0 = tile * P.bpt;
+        const int left = P.bands - t.bt.band0;
+        t.bt.nb = left < P.bpt ? left : P.bpt;
+        t.first = tile == tile0;
         t.last = tile + 1 == tile_end;
         return t;
     }
@@ -126,57 +142,10 @@ struct DtWalker {
     }
 };
 
-template <int WS, typename F>
-__device__ __forceinline__ void dt_runs(const TcDtParams& P, const DtTile& t, F&& f)
-{
-    const long long band_elems = (long long)WS * P.W;
-    long long g = t.band0;
-    const long long g_end = t.band0 + t.nb;
-    uint32_t soff = 0;
-    while (g < g_end) {
-        const long long b = g / P.nh;
-        const int i = (int)(g - b * P.nh);
-        long long run = P.nh - i;
-        if (run > g_end - g)
-            run = g_end - g;
-        const long long goff = ((b * P.C + t.c) * (long long)P.H + (long long)i * WS) * P.W;
-        const uint32_t bytes = (uint32_t)(run * band_elems * 2);
-        f(goff, soff, bytes);
-        soff += bytes;
-        g += run;
-    }
-}
-
-// One operand (rows = positions of `raw`, K = windows) -> K-major core matrices.
 template <int WS>
-__device__ __forceinline__ void dt_transform(const uint16_t* raw, uint8_t* dst, int nwin,
-                                             const int* woff, int W, int tw, int lane)
+__global__ void __launch_bounds__(kDtThreads, 1) wbmm_tc_dt_kernel(const __grid_constant__ TcDtParams P)
 {
-    using Cfg = DtCfg<WS>;
-    constexpr int NG = Cfg::NT / 8;
-    const int rl = lane & 7, pair = lane >> 3;
-#pragma unroll 1
-    for (int cm = tw; cm < Cfg::RG * NG; cm += 4) {
-        const int rg = cm / NG, ng = cm - (cm / NG) * NG;
-        const int row = rg * 8 + rl;
-        const int n0 = ng * 8 + pair * 2;
-        uint16_t lo = 0, hi = 0;
-        if (row < Cfg::D) {
-            const int pos = (row / WS) * W + (row - (row / WS) * WS);
-            if (n0 < nwin)
-                lo = raw[woff[n0] + pos];
-            if (n0 + 1 < nwin)
-                hi = raw[woff[n0 + 1] + pos];
-        }
-        *reinterpret_cast<uint32_t*>(dst + rg * Cfg::SBO + ng * 128 + rl * 16 + pair * 4) =
-            pack_bf16x2(lo, hi);
-    }
-}
-
-template <int WS>
-__global__ void __launch_bounds__(kDtThreads, 1) wbmm_tc_dt_kernel(const TcDtParams P)
-{
-    using Cfg = DtCfg<WS>;
+    using F = DtCfg<WS>;
     extern __shared__ __align__(1024) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     uint8_t* raw_base = smem + P.off_raw;
@@ -189,10 +158,10 @@ __global__ void __launch_bounds__(kDtThreads, 1) wbmm_tc_dt_kernel(const TcDtPar
     if (threadIdx.x == 0) {
         for (int i = 0; i < kDtRing; ++i) {
             mbar_init(&S.raw_full[i], 1);
-            mbar_init(&S.raw_empty[i], 4);
+            mbar_init(&S.raw_empty[i], kDtXformWarps);
         }
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&S.st_full[i], 4);
+            mbar_init(&S.st_full[i], kDtXformWarps);
             mbar_init(&S.st_empty[i], 1);
         }
         mbar_init(&S.g_full, 1);
@@ -201,10 +170,14 @@ __global__ void __launch_bounds__(kDtThreads, 1) wbmm_tc_dt_kernel(const TcDtPar
         S.abort = 0;
         fence_mbar_init();
     }
-    for (int n = threadIdx.x; n < Cfg::NT; n += kDtThreads) {
-        const int k = n / P.nw, j = n - (n / P.nw) * P.nw;
+    for (int n = threadIdx.x; n < F::NT; n += kDtThreads) {
+        const int k = n / P.nw, j = n - k * P.nw;
         woff[n] = k * WS * P.W + j * WS;
     }
+    // Operand stages start as zeros (padding slots are never written).
+    for (uint32_t e = threadIdx.x; e < 2 * F::STAGE_BYTES / 16; e += kDtThreads)
+        reinterpret_cast<uint4*>(st_base)[e] = make_uint4(0u, 0u, 0u, 0u);
+    fence_proxy_async_smem();
     if (warp == 1) {
         tmem_alloc(&S.tmem_slot, 512);
         tmem_relinquish();
@@ -216,26 +189,43 @@ __global__ void __launch_bounds__(kDtThreads, 1) wbmm_tc_dt_kernel(const TcDtPar
 
     if (warp == 0) {
         // ------------------------------------------------------ producer
-        if (lane == 0) {
-            int issued = 0, seq = 0;
-            DtWalker it;
-            for (it.start(P); it.valid(P); it.next(P), ++seq) {
-                const int s = seq % kDtRing;
-                if (*abort)
-                    break;
-                if (seq >= kDtRing && !mbar_wait(&S.raw_empty[s], ((seq / kDtRing) - 1) & 1,
-                                                 abort, P.budget, P.status))
-                    break;
-                const DtTile t = it.get(P);
-                const uint32_t bytes = (uint32_t)t.nb * WS * P.W * 2;
-                mbar_arrive_expect_tx(&S.raw_full[s], 2 * bytes);
-                uint8_t* slot = raw_base + (size_t)s * Cfg::RAW_BYTES;
-                dt_runs<WS>(P, t, [&](long long goff, uint32_t soff, uint32_t nbytes) {
-                    bulk_g2s(slot + soff, P.dy + goff, nbytes, &S.raw_full[s]);
-                    bulk_g2s(slot + Cfg::RAW_HALF + soff, P.x + goff, nbytes, &S.raw_full[s]);
-                });
+        // Lane 0 arms the slot's barrier; the lanes issue one run each.
+        int issued = 0, seq = 0;
+        DtWalker it;
+        for (it.start(P); it.valid(P); it.next(P), ++seq) {
+            const int s = seq % kDtRing;
+            bool ok = !*abort;
+            if (seq >= kDtRing)
+                ok = ok && mbar_wait(&S.raw_empty[s], ((seq / kDtRing) - 1) & 1, abort, P.budget,
+                                     P.status);
+            if (!__all_sync(0xffffffffu, ok))
+                break;
+            const DtTile t = it.get(P);
+            uint8_t* slot = raw_base + (size_t)s * F::RAW_BYTES;
+            if (P.use_tmap) {
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&S.raw_full[s], 2u * P.kimg * WS * P.W * P.nh * 2);
+                    tma_load_4d(slot, &P.map_dy, 0, 0, t.bt.c, t.bt.band0 / P.nh, &S.raw_full[s]);
+                    tma_load_4d(slot + F::RAW_HALF, &P.map_x, 0, 0, t.bt.c, t.bt.band0 / P.nh,
+                                &S.raw_full[s]);
+                }
                 issued = seq + 1;
+                continue;
             }
+            if (lane == 0)
+                mbar_arrive_expect_tx(&S.raw_full[s], 2u * t.bt.nb * WS * P.W * 2);
+            __syncwarp();
+            const BandRuns runs = band_runs(t.bt, P.nh);
+            for (int l = lane; l < runs.count; l += 32) {
+                long long goff;
+                uint32_t soff, nbytes;
+                band_run(t.bt, runs, l, WS, P.W, P.H, P.C, P.nh, goff, soff, nbytes);
+                bulk_g2s(slot + soff, P.dy + goff, nbytes, &S.raw_full[s]);
+                bulk_g2s(slot + F::RAW_HALF + soff, P.x + goff, nbytes, &S.raw_full[s]);
+            }
+            issued = seq + 1;
+        }
+        if (lane == 0) {
             for (int s = 0; s < kDtRing && s < issued; ++s) {
                 const int last = s + ((issued - 1 - s) / kDtRing) * kDtRing;
                 mbar_wait_drain(&S.raw_full[s], (last / kDtRing) & 1, P.budget, P.status);
@@ -251,23 +241,30 @@ __global__ void __launch_bounds__(kDtThreads, 1) wbmm_tc_dt_kernel(const TcDtPar
                 const DtTile t = it.get(P);
                 const int bs = seq & 1;
                 bool ok = !*abort;
-                if (t.first && item_seq > 0)
-                    ok = ok && mbar_wait(&S.g_empty, (item_seq - 1) & 1, abort, P.budget,
-                                         P.status);
+                if (t.first) {
+                    ok_item = true;
+                    if (item_seq > 0)
+                        ok = ok && mbar_wait(&S.g_empty, (item_seq - 1) & 1, abort, P.budget,
+                                             P.status);
+                }
                 ok = ok && mbar_wait(&S.st_full[bs], (seq >> 1) & 1, abort, P.budget, P.status);
-                ok_item = ok;
+                ok_item = ok_item && ok;
                 if (ok) {
                     tc_fence_after();
-                    const uint32_t a_addr = smem_u32(st_base + (size_t)bs * Cfg::STAGE_BYTES);
-                    const uint32_t b_addr = a_addr + Cfg::A_BYTES;
+                    const uint32_t a_addr = smem_u32(st_base + (size_t)bs * F::STAGE_BYTES);
+                    const uint32_t b_addr = a_addr + F::TILE_BYTES;
+                    const int nwin = t.bt.nb * P.nw;
+                    const int ksteps = (nwin + 15) >> 4;
 #pragma unroll
-                    for (int mt = 0; mt < Cfg::MT; ++mt) {
-#pragma unroll
-                        for (int k = 0; k < Cfg::KSTEPS; ++k) {
+                    for (int mt = 0; mt < F::MT; ++mt) {
+#pragma unroll 1
+                        for (int k = 0; k < ksteps; ++k) {
+                            // MN-major: LBO = window-group stride, SBO = position-group stride
                             const uint64_t adesc =
-                                smem_desc(a_addr + mt * 16 * Cfg::SBO + k * 256, 128, Cfg::SBO);
-                            const uint64_t bdesc = smem_desc(b_addr + k * 256, 128, Cfg::SBO);
-                            mma_ss(tmem + (uint32_t)(mt * 256), adesc, bdesc, Cfg::IDESC,
+                                smem_desc(a_addr + mt * 16 * 128 + k * 2 * F::SBO_T, F::SBO_T, 128);
+                            const uint64_t bdesc =
+                                smem_desc(b_addr + k * 2 * F::SBO_T, F::SBO_T, 128);
+                            mma_ss(tmem + (uint32_t)(mt * 256), adesc, bdesc, F::IDESC,
                                    (t.first && k == 0) ? 0u : 1u);
                         }
                     }
@@ -282,9 +279,9 @@ __global__ void __launch_bounds__(kDtThreads, 1) wbmm_tc_dt_kernel(const TcDtPar
             tc_commit(&S.fin);
             mbar_wait_drain(&S.fin, 0, P.budget, P.status);
         }
-    } else if (warp < 6) {
+    } else if (warp < kDtEpiWarp0) {
         // ------------------------------------------------------ transform
-        const int tw = warp - 2;
+        const int tt = threadIdx.x - 64;
         int seq = 0;
         DtWalker it;
         for (it.start(P); it.valid(P); it.next(P), ++seq) {
@@ -298,12 +295,14 @@ __global__ void __launch_bounds__(kDtThreads, 1) wbmm_tc_dt_kernel(const TcDtPar
             ok = __all_sync(0xffffffffu, ok);
             if (ok) {
                 const uint16_t* raw =
-                    reinterpret_cast<const uint16_t*>(raw_base + (size_t)s * Cfg::RAW_BYTES);
-                uint8_t* stage = st_base + (size_t)bs * Cfg::STAGE_BYTES;
-                const int nwin = t.nb * P.nw;
-                dt_transform<WS>(raw, stage, nwin, woff, P.W, tw, lane);
-                dt_transform<WS>(raw + Cfg::RAW_HALF / 2, stage + Cfg::A_BYTES, nwin, woff, P.W,
-                                 tw, lane);
+                    reinterpret_cast<const uint16_t*>(raw_base + (size_t)s * F::RAW_BYTES);
+                uint8_t* stage = st_base + (size_t)bs * F::STAGE_BYTES;
+                const int nwin = t.bt.nb * P.nw;
+                const int nzero = (nwin + 15) & ~15;    // last MMA K step reads up to here
+                transform_rows<WS>(raw, stage, F::SBO_T, nwin, nzero, woff, P.W, tt,
+                                   kDtXformWarps * 32);
+                transform_rows<WS>(raw + F::RAW_HALF / 2, stage + F::TILE_BYTES, F::SBO_T, nwin,
+                                   nzero, woff, P.W, tt, kDtXformWarps * 32);
                 fence_proxy_async_smem();
             }
             __syncwarp();
@@ -315,43 +314,94 @@ __global__ void __launch_bounds__(kDtThreads, 1) wbmm_tc_dt_kernel(const TcDtPar
     } else {
         // ------------------------------------------------------ epilogue
         const int quarter = warp & 3;
-        const int ew = warp - 6;
-        const int et = threadIdx.x - 6 * 32;
-        float* mybins = bins + ew * Cfg::TSZ;
+        const int ew = warp - kDtEpiWarp0;
+        const int et = threadIdx.x - kDtEpiWarp0 * 32;
+        float* mybins = bins + ew * F::TSZ;
         int item_seq = 0;
-        for (long long item = blockIdx.x; item < P.items; item += gridDim.x, ++item_seq) {
+        for (int item = blockIdx.x; item < P.items; item += gridDim.x, ++item_seq) {
             bool ok = !*abort;
             ok = ok && mbar_wait(&S.g_full, item_seq & 1, abort, P.budget, P.status);
             ok = __all_sync(0xffffffffu, ok);
             tc_fence_after();
-            for (int i = lane; i < Cfg::TSZ; i += 32)
+            for (int i = lane; i < F::TSZ; i += 32)
                 mybins[i] = 0.0f;
             __syncwarp();
             if (ok) {
+                // This warp reads rows u = mt*128 + quarter*32 + lane of G; with
+                // positions padded to RP slots per window row, the 32 lanes are
+                // 32/RP segments of one image row p each, and a 32-column TMEM
+                // chunk is 32/RP blocks of one column row r each.  The
+                // diagonal sums of a RP x RP block (fixed p, r) come from RP
+                // width-RP shuffles: lane L takes column s from lane (L+s)%RP,
+                // an entry of diagonal dq = L (no wrap) or dq = L - RP (wrap);
+                // fixed-shape tree sums give each lane the two diagonal sums of
+                // every block, kept in registers until the pass ends and then
+                // added to the bins of rows dp = p - r, one segment at a time.
+                constexpr int RP = F::RP;
+                constexpr int NB = 32 / RP;             // blocks (r values) per chunk
+                constexpr int NCH = (F::NPOS + 31) / 32;    // chunks per row (last may overhang)
+                const int L = lane & (RP - 1);
 #pragma unroll 1
-                for (int mt = 0; mt < Cfg::MT; ++mt) {
-                    const int u = mt * 128 + quarter * 32 + lane;
-                    const int p = u / WS, q = u - (u / WS) * WS;
-                    const int base = (p + WS - 1) * (2 * WS - 1) + (q + WS - 1);
+                for (int mt = 0; mt < F::MT; ++mt) {
+                    const int ubase = mt * 128 + quarter * 32;
+                    const int p = (ubase + lane) / RP;
+                    if (ubase / RP >= WS)
+                        break;                           // warp-uniform: only padding rows left
                     const uint32_t gcol =
                         tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(mt * 256);
-#pragma unroll 1
-                    for (int c0 = 0; c0 < Cfg::NP; c0 += 32) {
-                        uint32_t r[32];
-                        tmem_ld32(gcol + (uint32_t)c0, r);
-                        tmem_wait_ld(r);
-                        // Column v is the same for all lanes: lanes add into
-                        // distinct bins; __syncwarp orders columns.
+                    float dsum[WS][2];
 #pragma unroll
-                        for (int jj = 0; jj < 32; ++jj) {
-                            const int v = c0 + jj;
-                            if (v < Cfg::D && u < Cfg::D) {
-                                const int rr = v / WS, ss = v - (v / WS) * WS;
-                                const int bin = base - rr * (2 * WS - 1) - ss;
-                                mybins[bin] += __uint_as_float(r[jj]);
+                    for (int rr = 0; rr < WS; ++rr)
+                        dsum[rr][0] = dsum[rr][1] = 0.0f;
+                    uint32_t r[32];
+                    tmem_ld32(gcol, r);
+#pragma unroll
+                    for (int ch = 0; ch < NCH; ++ch) {
+                        tmem_wait_ld(r);
+                        float v[32];
+#pragma unroll
+                        for (int jj = 0; jj < 32; ++jj)
+                            v[jj] = __uint_as_float(r[jj]);
+                        if (ch + 1 < NCH)
+                            tmem_ld32(gcol + (uint32_t)((ch + 1) * 32), r);   // next chunk in flight
+#pragma unroll
+                        for (int b = 0; b < NB; ++b) {
+                            const int rr = ch * NB + b;
+                            if (rr < WS) {
+                                float a[RP], c[RP];
+#pragma unroll
+                                for (int s = 0; s < RP; ++s) {
+                                    const float g = __shfl_sync(0xffffffffu, v[b * RP + s],
+                                                                (L + s) & (RP - 1), RP);
+                                    const bool in_a = L + s < RP;
+                                    a[s] = in_a ? g : 0.0f;
+                                    c[s] = in_a ? 0.0f : g;
+                                }
+#pragma unroll
+                                for (int h = RP / 2; h >= 1; h /= 2)
+#pragma unroll
+                                    for (int s = 0; s < h; ++s) {
+                                        a[s] = a[s] + a[s + h];
+                                        c[s] = c[s] + c[s + h];
+                                    }
+                                dsum[rr][0] = a[0];
+                                dsum[rr][1] = c[0];
                             }
-                            __syncwarp();
                         }
+                    }
+#pragma unroll
+                    for (int seg = 0; seg < 32 / RP; ++seg) {
+                        if (lane / RP == seg && p < WS) {
+#pragma unroll
+                            for (int rr = 0; rr < WS; ++rr) {
+                                const int row = (p - rr + WS - 1) * (2 * WS - 1) + (WS - 1);
+                                if (L <= WS - 1)
+                                    mybins[row + L] += dsum[rr][0];
+                                if (L - RP >= -(WS - 1))
+                                    mybins[row + L - RP] += dsum[rr][1];
+                            }
+                        }
+                        __syncwarp();
                     }
                 }
             }
@@ -361,12 +411,12 @@ __global__ void __launch_bounds__(kDtThreads, 1) wbmm_tc_dt_kernel(const TcDtPar
                 mbar_arrive(&S.g_empty);
             named_bar_sync(3, 128);
             if (ok) {
-                float* out = P.partials + item * Cfg::TSZ;
-                for (int i = et; i < Cfg::TSZ; i += 128) {
+                float* out = P.partials + (long long)item * F::TSZ;
+                for (int i = et; i < F::TSZ; i += 128) {
                     float acc = bins[i];
-                    acc += bins[Cfg::TSZ + i];
-                    acc += bins[2 * Cfg::TSZ + i];
-                    acc += bins[3 * Cfg::TSZ + i];
+                    acc += bins[F::TSZ + i];
+                    acc += bins[2 * F::TSZ + i];
+                    acc += bins[3 * F::TSZ + i];
                     out[i] = acc;
                 }
             }
@@ -386,7 +436,6 @@ __global__ void __launch_bounds__(kDtThreads, 1) wbmm_tc_dt_kernel(const TcDtPar
 // ------------------------------------------------------------------ host
 namespace {
 
-constexpr uint32_t kSmemMax = 232448;
 constexpr uint32_t kMinSmem = 120 * 1024;
 inline uint32_t align_up(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
 
@@ -397,38 +446,40 @@ struct DtLayout {
 template <int WS>
 DtLayout dt_layout()
 {
-    using Cfg = DtCfg<WS>;
+    using F = DtCfg<WS>;
     DtLayout L;
     uint32_t off = 0;
     L.off_stage = off;
-    off += 2 * Cfg::STAGE_BYTES;
+    off += 2 * F::STAGE_BYTES;
     L.off_raw = align_up(off, 128);
-    off = L.off_raw + kDtRing * Cfg::RAW_BYTES;
+    off = L.off_raw + kDtRing * F::RAW_BYTES;
     L.off_bins = align_up(off, 16);
-    off = L.off_bins + 4 * Cfg::TSZ * 4;
+    off = L.off_bins + 4 * F::TSZ * 4;
     L.off_woff = align_up(off, 16);
-    off = L.off_woff + Cfg::NT * 4;
+    off = L.off_woff + F::NT * 4;
     L.off_bar = align_up(off, 16);
     off = L.off_bar + sizeof(DtBars);
     L.total = align_up(off, 1024);
-    // at least half the SM's shared memory: one CTA (and one 512-column
-    // TMEM allocation) per SM
+    // at least half the SM's shared memory: one CTA (and one 512-column TMEM
+    // allocation) per SM
     if (L.total < kMinSmem)
         L.total = kMinSmem;
     return L;
 }
 
-// Tiles per chunk: a fixed function of the shape (never of the grid).
+// Tiles per chunk: a fixed function of the shape (never of the grid).  Each
+// chunk ends with one reduction of G, so chunks are as long as the channel
+// allows, up to 16 tiles.
 int chunk_tiles(int tpc)
 {
-    return tpc < 2 ? 1 : 2;
+    return tpc < 16 ? tpc : 16;
 }
 
 template <int WS>
 cudaError_t dt_launch_ws(const Geom& g, const void* x, const void* dy, float* partials,
                          const Launch& L)
 {
-    using Cfg = DtCfg<WS>;
+    using F = DtCfg<WS>;
     const DtLayout lay = dt_layout<WS>();
     if (lay.total > kSmemMax)
         return cudaErrorInvalidConfiguration;
@@ -448,22 +499,31 @@ cudaError_t dt_launch_ws(const Geom& g, const void* x, const void* dy, float* pa
     P.dy = static_cast<const uint16_t*>(dy);
     P.partials = partials;
     P.C = g.C; P.H = g.H; P.W = g.W; P.nh = g.nh; P.nw = g.nw;
-    P.bpt = Cfg::NT / g.nw;
-    P.bands = g.bands;
-    P.tpc = (int)((g.bands + P.bpt - 1) / P.bpt);
+    P.bpt = F::NT / g.nw;
+    P.bands = (int)g.bands;
+    P.tpc = (P.bands + P.bpt - 1) / P.bpt;
     P.ch = chunk_tiles(P.tpc);
     P.chunks = (P.tpc + P.ch - 1) / P.ch;
-    P.items = (long long)g.C * P.chunks;
+    P.items = g.C * P.chunks;
+    P.use_tmap = 0;
+    P.kimg = 0;
+    if (P.bpt % g.nh == 0) {
+        const int k = P.bpt / g.nh;
+        if (encode_plane_map(&P.map_x, x, g, k) && encode_plane_map(&P.map_dy, dy, g, k)) {
+            P.use_tmap = 1;
+            P.kimg = k;
+        }
+    }
     P.off_raw = lay.off_raw; P.off_stage = lay.off_stage; P.off_bins = lay.off_bins;
     P.off_woff = lay.off_woff; P.off_bar = lay.off_bar;
     P.budget = L.budget;
     P.status = L.status;
-    long long grid = L.num_sms;
+    int grid = L.num_sms;
     if (grid > P.items)
         grid = P.items;
     if (grid < 1)
         return cudaSuccess;
-    wbmm_tc_dt_kernel<WS><<<(unsigned)grid, kDtThreads, lay.total, L.stream>>>(P);
+    wbmm_tc_dt_kernel<WS><<<grid, kDtThreads, lay.total, L.stream>>>(P);
     note_launches(1);
     return cudaGetLastError();
 }
@@ -474,16 +534,18 @@ bool tc_dt_supported(const Geom& g)
 {
     if (g.w < 2 || g.w > 16)
         return false;
-    if (g.nw > 64)
+    if (g.nw > dt_nt_for(g.w))
         return false;
     if (((long long)g.w * g.W * 2) % 16 != 0)
+        return false;
+    if (g.bands * (long long)g.C >= (1ll << 31))
         return false;
     return true;
 }
 
 int tc_dt_chunks(const Geom& g)
 {
-    const int bpt = 64 / g.nw;
+    const int bpt = dt_nt_for(g.w) / g.nw;
     const int tpc = (int)((g.bands + bpt - 1) / bpt);
     const int ch = chunk_tiles(tpc);
     return (tpc + ch - 1) / ch;

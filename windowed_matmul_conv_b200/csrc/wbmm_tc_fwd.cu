@@ -6,62 +6,78 @@
 // memory once; it is the A operand of every MMA of that channel and is never
 // written to HBM.  Windows stream through as the GEMM's N dimension:
 //
-//   D[u, n] = sum_v A[u, v] * X[v, n]        u, v in-window positions,
-//                                            n the windows of the tile
+//   D[u, n] = sum_k A[u, k] * X[k, n]     u = p*w+q output position (lane),
+//                                         k = r*RP+s padded input position,
+//                                         n the windows of the tile
 //
-// Warp roles (320 threads):
-//   warp 0      producer: bulk-copies the tile's bands (contiguous NCHW
-//               strips, w rows x W) into a ring of raw shared-memory slots
-//   warp 1      MMA issuer (one thread) and TMEM owner
-//   warps 2..5  transform: raw band layout -> K-major UMMA operand (no
-//               swizzle, 8x16B core matrices); on a channel change they
-//               expand the table (or load the cached matrix) into TMEM
-//   warps 6..9  epilogue: TMEM -> registers -> bf16 (round to nearest even)
-//               -> band layout in shared memory -> bulk store to NCHW
+// Warp roles (640 threads):
+//   warp 0        producer: bulk-copies the tile's bands (contiguous NCHW
+//                 strips, w rows x W) into a ring of raw shared-memory
+//                 slots, one run of bands per lane
+//   warp 1        MMA issuer (one thread) and TMEM owner
+//   warp 2        storer: bulk-stores finished output slots to NCHW
+//   warps 3..7    transform: raw band layout -> K-major operand, one window
+//                 row per thread as whole 16-byte core-matrix rows
+//   warps 8..11   A builders: on a channel change they write M_c into TMEM,
+//                 one tcgen05.st per (row u, window row r) from contiguous
+//                 table slices; loads and transforms keep running meanwhile
+//   warps 12..19  epilogue: TMEM -> registers -> bf16 (round to nearest
+//                 even) -> band layout in shared memory
 //
-// Pipeline: raw ring (R slots) -> operand stages (2) -> accumulators (2).
+// Pipeline: raw ring (R slots) -> operand stages (2) -> accumulators (2)
+// -> output slots (2).
 // Every wait is bounded; a wait that runs out raises the CTA's abort flag and
 // the device status word, and every role then runs its loop without doing
 // work so that all threads reach the drain and the TMEM release.
 #include <cuda_bf16.h>
 
 #include "ptx_sm100.cuh"
+#include "tc_common.cuh"
 #include "wbmm_internal.h"
 
 namespace wbmm {
 
 template <int WS>
-struct FwdCfg {
-    static constexpr int D = WS * WS;
-    static constexpr int KP = (D + 15) / 16 * 16;          // K padded to the MMA K step
-    static constexpr int MT = (D + 127) / 128;             // 128-row M tiles
+struct FwdCfg : PadCfg<WS> {
+    using P = PadCfg<WS>;
+    static constexpr int MT = (P::D + 127) / 128;          // 128-row M tiles
     static constexpr int NT = (MT == 1) ? 128 : 64;        // windows per tile (MMA N)
-    static constexpr int KSTEPS = KP / 16;
-    static constexpr int TSZ = (2 * WS - 1) * (2 * WS - 1);
-    static constexpr int A_COLS = MT * KP / 2;             // TMEM columns of bf16 pairs
+    static constexpr int KSTEPS = P::KP / 16;
+    static constexpr int A_COLS = MT * P::KP / 2;          // TMEM columns of bf16 pairs
     static constexpr int D_COL0 = 256;                     // accumulators at [256, 512)
-    static constexpr uint32_t RAW_BYTES = (uint32_t)((NT * D * 2 + 127) / 128 * 128);
-    static constexpr uint32_t B_BYTES = (uint32_t)(NT * KP * 2);
-    static constexpr uint32_t SBO_B = (uint32_t)(KP * 16);  // bytes per 8-window group
-    static constexpr uint32_t TBL_BYTES = (uint32_t)((TSZ * 2 + 15) / 16 * 16);
+    static constexpr uint32_t RAW_BYTES = (uint32_t)((NT * P::D * 2 + 127) / 128 * 128);
+    static constexpr uint32_t B_BYTES = (uint32_t)(NT * P::KP * 2);
+    static constexpr uint32_t SBO_B = (uint32_t)(P::KP * 16);   // bytes per 8-window group
+    static constexpr int TROW = 2 * WS;                          // table copy row stride
+    static constexpr uint32_t TCOPY_BYTES = (uint32_t)(((2 * WS - 1) * TROW * 2 + 15) / 16 * 16);
     static constexpr uint32_t IDESC = idesc_bf16(128, NT);
     static_assert(A_COLS <= D_COL0, "A operand must fit below the accumulators");
     static_assert(2 * MT * NT <= 256, "two accumulators must fit in 256 columns");
 };
 
 constexpr int kMaxRing = 8;
-constexpr int kThreads = 320;
+// warp roles: 0 producer, 1 MMA, 2 storer, 3..7 transform, 8..11 A builders,
+// 12..19 epilogue
+constexpr int kTransformWarps = 5;
+constexpr int kBuildWarp0 = 3 + kTransformWarps;
+constexpr int kEpiWarp0 = kBuildWarp0 + 4;
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = (kEpiWarp0 + kEpiWarps) * 32;
 
 struct TcFwdParams {
+    TmapBytes map_x;        // whole-plane tensor maps (used when use_tmap)
+    TmapBytes map_y;
     const uint16_t* x;      // bf16 bits, [B][C][H][W]
     const uint16_t* src;    // table [C][tsz] or matrices [C][d][d]
     uint16_t* y;            // output map
     int C, H, W, nh, nw;
     int bpt;                // bands per tile
     int tpc;                // tiles per channel
-    long long bands;        // bands per channel
-    long long items;        // C * tpc
+    int bands;              // bands per channel
+    int items;              // C * tpc
     int R;                  // raw ring depth
+    int use_tmap;           // tiles are whole planes: one 4-D TMA per tile
+    int kimg;               // planes per tile (bpt / nh) when use_tmap
     uint32_t off_raw, off_b, off_out, off_tbl, off_woff, off_bar;
     unsigned long long budget;
     int* status;
@@ -74,6 +90,8 @@ struct Bars {
     uint64_t b_empty[2];
     uint64_t acc_full[2];
     uint64_t acc_empty[2];
+    uint64_t out_full[2];
+    uint64_t out_empty[2];
     uint64_t a_full;
     uint64_t a_empty;
     uint64_t fin;
@@ -81,165 +99,136 @@ struct Bars {
     int abort;
 };
 
-struct TileRef {
-    int c;
-    long long band0;
-    int nb;
-};
-
-__device__ __forceinline__ TileRef tile_ref(const TcFwdParams& P, long long it)
+__device__ __forceinline__ BandTile tile_of(const TcFwdParams& P, int it)
 {
-    TileRef t;
-    t.c = (int)(it / P.tpc);
-    const int ti = (int)(it - (long long)t.c * P.tpc);
-    t.band0 = (long long)ti * P.bpt;
-    const long long left = P.bands - t.band0;
-    t.nb = (int)(left < P.bpt ? left : P.bpt);
+    BandTile t;
+    t.c = it / P.tpc;
+    t.band0 = (it - t.c * P.tpc) * P.bpt;
+    const int left = P.bands - t.band0;
+    t.nb = left < P.bpt ? left : P.bpt;
     return t;
 }
 
-// Calls f(global element offset, byte offset in the slot, bytes) for each
-// contiguous run of bands (bands of one image plane are adjacent in NCHW).
-template <int WS, typename F>
-__device__ __forceinline__ void for_each_run(const TcFwdParams& P, const TileRef& t, F&& f)
+// Loads the table rows the A builders slice from: copy 0 is the source table
+// with rows padded to 2w entries, copy 1 the same shifted left by one entry,
+// so a slice starting at any column is read as aligned 32-bit words.  The
+// forward (M_c[u][v]) reads rows reversed; the input gradient (M_c[v][u])
+// reads them as stored.
+template <int WS, int MODE>
+__device__ __forceinline__ void load_tables(uint16_t* c0, uint16_t* c1, const uint16_t* T,
+                                            int tid, int nthreads)
 {
-    const long long band_elems = (long long)WS * P.W;
-    long long g = t.band0;
-    const long long g_end = t.band0 + t.nb;
-    uint32_t soff = 0;
-    while (g < g_end) {
-        const long long b = g / P.nh;
-        const int i = (int)(g - b * P.nh);
-        long long run = P.nh - i;
-        if (run > g_end - g)
-            run = g_end - g;
-        const long long goff = ((b * P.C + t.c) * (long long)P.H + (long long)i * WS) * P.W;
-        const uint32_t bytes = (uint32_t)(run * band_elems * 2);
-        f(goff, soff, bytes);
-        soff += bytes;
-        g += run;
+    using F = FwdCfg<WS>;
+    constexpr int L = 2 * WS - 1;
+    for (int e = tid; e < L * F::TROW; e += nthreads) {
+        const int a = e / F::TROW, col = e - a * F::TROW;
+        auto src = [&](int cc) -> uint16_t {
+            if (cc >= L)
+                return 0;
+            return T[a * L + (MODE == kTable ? (L - 1 - cc) : cc)];
+        };
+        c0[e] = src(col);
+        c1[e] = src(col + 1);
     }
 }
 
-// Relative-table entry of M_c[u][v] (or of M_c[v][u] when flipped).
+// Writes this warp's 32 lanes (rows u) of the A operand into TMEM: for each
+// window row r the RP/2 columns holding slots r*RP .. r*RP+RP-1.
 template <int WS, int MODE>
-__device__ __forceinline__ uint16_t a_elem(const uint16_t* tbl, const uint16_t* Mc, int u, int p,
-                                           int q, int v)
+__device__ __forceinline__ void build_a(uint32_t tmem, const uint16_t* c0, const uint16_t* c1,
+                                        const uint16_t* Mc, int quarter, int lane)
 {
-    constexpr int D = WS * WS;
-    constexpr int TSZ = (2 * WS - 1) * (2 * WS - 1);
-    if (v >= D)
-        return 0;
-    if (MODE == kCached)
-        return Mc[(long long)u * D + v];
-    const int r = v / WS, s = v - (v / WS) * WS;
-    const int idx = (p - r + WS - 1) * (2 * WS - 1) + (q - s + WS - 1);
-    return tbl[MODE == kTableFlip ? (TSZ - 1 - idx) : idx];
-}
-
-// Writes the A operand (rows u = lanes, K pairs packed in 32-bit columns)
-// of this warp's 32-lane quarter into TMEM.
-template <int WS, int MODE>
-__device__ __forceinline__ void expand_a(uint32_t tmem, const uint16_t* tbl, const uint16_t* Mc,
-                                         int quarter, int lane)
-{
-    using Cfg = FwdCfg<WS>;
+    using F = FwdCfg<WS>;
 #pragma unroll 1
-    for (int mt = 0; mt < Cfg::MT; ++mt) {
+    for (int mt = 0; mt < F::MT; ++mt) {
         const int u = mt * 128 + quarter * 32 + lane;
-        const bool uval = u < Cfg::D;
-        const int p = u / WS, q = u - (u / WS) * WS;
+        const bool uval = u < F::D;
+        const int p = uval ? u / WS : 0, q = uval ? u - (u / WS) * WS : 0;
+        const int col0 = WS - 1 - q;                       // first table column of a slice
+        const uint16_t* tcopy = (col0 & 1) ? c1 : c0;
+        const int cbase = col0 & ~1;
+        const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(mt * (F::KP / 2));
 #pragma unroll 1
-        for (int c8 = 0; c8 < Cfg::KP / 2; c8 += 8) {
-            uint32_t r[8];
+        for (int r = 0; r < WS; ++r) {
+            uint32_t wv[F::RP / 2];
+            if (MODE == kCached) {
+                const uint16_t* row = Mc + (long long)u * F::D + r * WS;
 #pragma unroll
-            for (int jj = 0; jj < 8; ++jj) {
-                const int v0 = 2 * (c8 + jj);
-                uint16_t lo = 0, hi = 0;
-                if (uval) {
-                    lo = a_elem<WS, MODE>(tbl, Mc, u, p, q, v0);
-                    hi = a_elem<WS, MODE>(tbl, Mc, u, p, q, v0 + 1);
-                }
-                r[jj] = pack_bf16x2(lo, hi);
-            }
-            tmem_st8(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(mt * (Cfg::KP / 2) + c8),
-                     r);
-        }
-    }
-}
-
-// Raw band layout -> K-major operand.  One warp instruction writes one
-// 8-window x 8-position core matrix (128 contiguous bytes, conflict free).
-template <int WS>
-__device__ __forceinline__ void transform_tile(const uint16_t* raw, uint8_t* bst, int nwin,
-                                               const int* woff, int W, int tw, int lane)
-{
-    using Cfg = FwdCfg<WS>;
-    constexpr int KG = Cfg::KP / 8;
-    constexpr int NG = Cfg::NT / 8;
-    const int nl = lane & 7, pair = lane >> 3;
-#pragma unroll 1
-    for (int g8 = tw; g8 < NG; g8 += 4) {
-        if (g8 * 8 >= nwin)
-            break;
-        const int n = g8 * 8 + nl;
-        const bool nval = n < nwin;
-        const int wo = nval ? woff[n] : 0;
-        uint32_t* dst = reinterpret_cast<uint32_t*>(bst + g8 * Cfg::SBO_B + nl * 16 + pair * 4);
-#pragma unroll 2
-        for (int vg = 0; vg < KG; ++vg) {
-            const int v = vg * 8 + pair * 2;
-            uint32_t word = 0;
-            if (nval && v < Cfg::D) {
-                if (WS % 2 == 0) {
-                    const int r = v / WS, s = v - (v / WS) * WS;
-                    word = *reinterpret_cast<const uint32_t*>(raw + wo + r * W + s);
-                } else {
-                    const int r0 = v / WS, s0 = v - r0 * WS;
-                    const uint16_t lo = raw[wo + r0 * W + s0];
-                    uint16_t hi = 0;
-                    if (v + 1 < Cfg::D) {
-                        const int r1 = (v + 1) / WS, s1 = (v + 1) - r1 * WS;
-                        hi = raw[wo + r1 * W + s1];
+                for (int m = 0; m < F::RP / 2; ++m) {
+                    uint32_t v = 0;
+                    if (uval && 2 * m < WS) {
+                        if (WS % 2 == 0) {
+                            v = __ldg(reinterpret_cast<const unsigned int*>(row) + m);
+                        } else {
+                            const uint16_t lo = row[2 * m];
+                            const uint16_t hi = (2 * m + 1 < WS) ? row[2 * m + 1] : (uint16_t)0;
+                            v = pack_bf16x2(lo, hi);
+                        }
                     }
-                    word = pack_bf16x2(lo, hi);
+                    wv[m] = v;
+                }
+            } else {
+                const int a = (MODE == kTable) ? (p - r + WS - 1) : (r - p + WS - 1);
+                const uint32_t* srow =
+                    reinterpret_cast<const uint32_t*>(tcopy + a * F::TROW + cbase);
+#pragma unroll
+                for (int m = 0; m < F::RP / 2; ++m) {
+                    uint32_t v = (uval && 2 * m < WS) ? srow[m] : 0u;
+                    if (WS % 2 == 1 && 2 * m + 1 == WS)
+                        v &= 0xFFFFu;
+                    wv[m] = v;
                 }
             }
-            dst[vg * 32] = word;
+            if constexpr (F::RP == 16) {
+                tmem_st8(taddr + (uint32_t)(r * 8), wv);
+            } else {
+                tmem_st4(taddr + (uint32_t)(r * 4), wv);
+            }
+        }
+        if (F::KP > F::K) {
+            // zero the K columns past the last window row (odd small w)
+            const uint32_t z[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+            for (int cc = F::K / 2; cc < F::KP / 2; cc += 4)
+                tmem_st4(taddr + (uint32_t)cc, z);
         }
     }
 }
 
 template <int WS, int MODE>
-__global__ void __launch_bounds__(kThreads, 1) wbmm_tc_fwd_kernel(const TcFwdParams P)
+__global__ void __launch_bounds__(kThreads, 1) wbmm_tc_fwd_kernel(const __grid_constant__ TcFwdParams P)
 {
-    using Cfg = FwdCfg<WS>;
+    using F = FwdCfg<WS>;
     extern __shared__ __align__(1024) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     uint8_t* raw_base = smem + P.off_raw;
     uint8_t* b_base = smem + P.off_b;
     uint8_t* out_base = smem + P.off_out;
+    uint16_t* tc0 = reinterpret_cast<uint16_t*>(smem + P.off_tbl);
+    uint16_t* tc1 = reinterpret_cast<uint16_t*>(smem + P.off_tbl + F::TCOPY_BYTES);
     int* woff = reinterpret_cast<int*>(smem + P.off_woff);
     Bars& S = *reinterpret_cast<Bars*>(smem + P.off_bar);
     volatile int* abort = &S.abort;
     const int R = P.R;
 
     // Contiguous, balanced range of items for this CTA.
-    const long long q = P.items / gridDim.x, rem = P.items % gridDim.x;
-    const long long it0 = blockIdx.x * q + (blockIdx.x < rem ? blockIdx.x : rem);
-    const int n_it = (int)(q + (blockIdx.x < rem ? 1 : 0));
+    const int q = P.items / (int)gridDim.x, rem = P.items % (int)gridDim.x;
+    const int it0 = (int)blockIdx.x * q + ((int)blockIdx.x < rem ? (int)blockIdx.x : rem);
+    const int n_it = q + ((int)blockIdx.x < rem ? 1 : 0);
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kMaxRing; ++i) {
             mbar_init(&S.raw_full[i], 1);
-            mbar_init(&S.raw_empty[i], 4);
+            mbar_init(&S.raw_empty[i], kTransformWarps);
         }
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&S.b_full[i], 4);
+            mbar_init(&S.b_full[i], kTransformWarps);
             mbar_init(&S.b_empty[i], 1);
             mbar_init(&S.acc_full[i], 1);
-            mbar_init(&S.acc_empty[i], 4);
+            mbar_init(&S.acc_empty[i], kEpiWarps);
+            mbar_init(&S.out_full[i], kEpiWarps);
+            mbar_init(&S.out_empty[i], 1);
         }
         mbar_init(&S.a_full, 4);
         mbar_init(&S.a_empty, 1);
@@ -247,10 +236,15 @@ __global__ void __launch_bounds__(kThreads, 1) wbmm_tc_fwd_kernel(const TcFwdPar
         S.abort = 0;
         fence_mbar_init();
     }
-    for (int n = threadIdx.x; n < Cfg::NT; n += kThreads) {
-        const int k = n / P.nw, j = n - (n / P.nw) * P.nw;
+    for (int n = threadIdx.x; n < F::NT; n += kThreads) {
+        const int k = n / P.nw, j = n - k * P.nw;
         woff[n] = k * WS * P.W + j * WS;
     }
+    // Operand stages start as zeros: K slots past the last window row are
+    // never written by the transform.
+    for (uint32_t e = threadIdx.x; e < 2 * F::B_BYTES / 16; e += kThreads)
+        reinterpret_cast<uint4*>(b_base)[e] = make_uint4(0u, 0u, 0u, 0u);
+    fence_proxy_async_smem();
     if (warp == 1) {
         tmem_alloc(&S.tmem_slot, 512);
         tmem_relinquish();
@@ -262,25 +256,42 @@ __global__ void __launch_bounds__(kThreads, 1) wbmm_tc_fwd_kernel(const TcFwdPar
 
     if (warp == 0) {
         // ------------------------------------------------------ producer
-        if (lane == 0) {
-            int issued = 0;
-            for (int seq = 0; seq < n_it; ++seq) {
-                const int s = seq % R;
-                if (*abort)
-                    break;
-                if (seq >= R && !mbar_wait(&S.raw_empty[s], ((seq / R) - 1) & 1, abort, P.budget,
-                                           P.status))
-                    break;
-                const TileRef t = tile_ref(P, it0 + seq);
-                const uint32_t bytes = (uint32_t)t.nb * WS * P.W * 2;
-                mbar_arrive_expect_tx(&S.raw_full[s], bytes);
-                uint8_t* slot = raw_base + (size_t)s * Cfg::RAW_BYTES;
-                for_each_run<WS>(P, t, [&](long long goff, uint32_t soff, uint32_t nbytes) {
-                    bulk_g2s(slot + soff, P.x + goff, nbytes, &S.raw_full[s]);
-                });
+        // Lane 0 arms the slot's barrier; the lanes issue one run each.
+        int issued = 0;
+        for (int seq = 0; seq < n_it; ++seq) {
+            const int s = seq % R;
+            bool ok = !*abort;
+            if (seq >= R)
+                ok = ok && mbar_wait(&S.raw_empty[s], ((seq / R) - 1) & 1, abort, P.budget,
+                                     P.status);
+            if (!__all_sync(0xffffffffu, ok))
+                break;
+            const BandTile t = tile_of(P, it0 + seq);
+            uint8_t* slot = raw_base + (size_t)s * F::RAW_BYTES;
+            if (P.use_tmap) {
+                // whole planes: one request; a box past the last image is
+                // zero-filled and still counts its full size
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&S.raw_full[s], (uint32_t)P.kimg * WS * P.W * P.nh * 2);
+                    tma_load_4d(slot, &P.map_x, 0, 0, t.c, t.band0 / P.nh, &S.raw_full[s]);
+                }
                 issued = seq + 1;
+                continue;
             }
-            // Drain: every issued copy lands before the CTA can exit.
+            if (lane == 0)
+                mbar_arrive_expect_tx(&S.raw_full[s], (uint32_t)t.nb * WS * P.W * 2);
+            __syncwarp();
+            const BandRuns runs = band_runs(t, P.nh);
+            for (int l = lane; l < runs.count; l += 32) {
+                long long goff;
+                uint32_t soff, nbytes;
+                band_run(t, runs, l, WS, P.W, P.H, P.C, P.nh, goff, soff, nbytes);
+                bulk_g2s(slot + soff, P.x + goff, nbytes, &S.raw_full[s]);
+            }
+            issued = seq + 1;
+        }
+        // Drain: every issued copy lands before the CTA can exit.
+        if (lane == 0) {
             for (int s = 0; s < R && s < issued; ++s) {
                 const int last = s + ((issued - 1 - s) / R) * R;
                 mbar_wait_drain(&S.raw_full[s], (last / R) & 1, P.budget, P.status);
@@ -291,7 +302,7 @@ __global__ void __launch_bounds__(kThreads, 1) wbmm_tc_fwd_kernel(const TcFwdPar
         if (lane == 0) {
             int cur_c = -1, ci = 0;
             for (int seq = 0; seq < n_it; ++seq) {
-                const TileRef t = tile_ref(P, it0 + seq);
+                const BandTile t = tile_of(P, it0 + seq);
                 bool ok = !*abort;
                 if (t.c != cur_c) {
                     ok = ok && mbar_wait(&S.a_full, ci & 1, abort, P.budget, P.status);
@@ -306,22 +317,23 @@ __global__ void __launch_bounds__(kThreads, 1) wbmm_tc_fwd_kernel(const TcFwdPar
                 if (!ok)
                     continue;
                 tc_fence_after();
-                const uint32_t b_addr = smem_u32(b_base + (size_t)bs * Cfg::B_BYTES);
+                // Descriptors differ per K step only in the start-address
+                // field (+256 bytes = +16 in 16-byte units); the loop is fully
+                // unrolled so each MMA issues with a couple of integer adds.
+                const uint64_t bdesc0 =
+                    smem_desc(smem_u32(b_base + (size_t)bs * F::B_BYTES), 128, F::SBO_B);
+                const uint32_t d0 = tmem + F::D_COL0 + (uint32_t)(ab * F::MT * F::NT);
 #pragma unroll
-                for (int mt = 0; mt < Cfg::MT; ++mt) {
-                    const uint32_t d_tmem =
-                        tmem + Cfg::D_COL0 + (uint32_t)(ab * Cfg::MT * Cfg::NT + mt * Cfg::NT);
-                    const uint32_t a_tmem = tmem + (uint32_t)(mt * (Cfg::KP / 2));
-#pragma unroll 1
-                    for (int k = 0; k < Cfg::KSTEPS; ++k) {
-                        const uint64_t bdesc = smem_desc(b_addr + k * 256, 128, Cfg::SBO_B);
-                        mma_ts(d_tmem, a_tmem + (uint32_t)(k * 8), bdesc, Cfg::IDESC, k > 0);
-                    }
+                for (int mt = 0; mt < F::MT; ++mt) {
+#pragma unroll
+                    for (int k = 0; k < F::KSTEPS; ++k)
+                        mma_ts(d0 + (uint32_t)(mt * F::NT), tmem + (uint32_t)(mt * (F::KP / 2) + k * 8),
+                               bdesc0 + (uint64_t)(k * 16), F::IDESC, k > 0 ? 1u : 0u);
                 }
                 tc_commit(&S.b_empty[bs]);
                 tc_commit(&S.acc_full[ab]);
                 const bool last_of_channel =
-                    (seq == n_it - 1) || (tile_ref(P, it0 + seq + 1).c != t.c);
+                    (seq == n_it - 1) || (tile_of(P, it0 + seq + 1).c != t.c);
                 if (last_of_channel)
                     tc_commit(&S.a_empty);
             }
@@ -329,39 +341,40 @@ __global__ void __launch_bounds__(kThreads, 1) wbmm_tc_fwd_kernel(const TcFwdPar
             tc_commit(&S.fin);
             mbar_wait_drain(&S.fin, 0, P.budget, P.status);
         }
-    } else if (warp < 6) {
-        // ------------------------------------------------------ transform
-        const int tw = warp - 2;
-        const int quarter = warp & 3;
-        uint16_t* tbl = reinterpret_cast<uint16_t*>(smem + P.off_tbl + tw * Cfg::TBL_BYTES);
-        int cur_c = -1, ci = 0;
+    } else if (warp == 2) {
+        // ------------------------------------------------------ storer
+        // Bulk-stores each finished output slot (one run per lane), waits
+        // until the copies have read shared memory, then frees the slot.
         for (int seq = 0; seq < n_it; ++seq) {
-            const TileRef t = tile_ref(P, it0 + seq);
-            if (t.c != cur_c) {
-                bool ok = !*abort;
-                if (ci > 0)
-                    ok = ok && mbar_wait(&S.a_empty, (ci - 1) & 1, abort, P.budget, P.status);
-                ok = __all_sync(0xffffffffu, ok);
-                tc_fence_after();
-                const uint16_t* Mc = nullptr;
-                if (MODE == kCached) {
-                    Mc = P.src + (long long)t.c * Cfg::D * Cfg::D;
-                } else {
-                    for (int i = lane; i < Cfg::TSZ; i += 32)
-                        tbl[i] = P.src[(long long)t.c * Cfg::TSZ + i];
-                    __syncwarp();
+            const int os = seq & 1;
+            bool ok = !*abort;
+            ok = ok && mbar_wait(&S.out_full[os], (seq >> 1) & 1, abort, P.budget, P.status);
+            ok = __all_sync(0xffffffffu, ok);
+            if (ok) {
+                const BandTile t = tile_of(P, it0 + seq);
+                const BandRuns runs = band_runs(t, P.nh);
+                const uint8_t* out = out_base + (size_t)os * F::RAW_BYTES;
+                if (P.use_tmap && lane == 0)       // planes past the last image are clipped
+                    tma_store_4d(&P.map_y, 0, 0, t.c, t.band0 / P.nh, out);
+                for (int l = P.use_tmap ? runs.count : lane; l < runs.count; l += 32) {
+                    long long goff;
+                    uint32_t soff, nbytes;
+                    band_run(t, runs, l, WS, P.W, P.H, P.C, P.nh, goff, soff, nbytes);
+                    bulk_s2g(P.y + goff, out + soff, nbytes);
                 }
-                if (ok) {
-                    expand_a<WS, MODE>(tmem, tbl, Mc, quarter, lane);
-                    tmem_wait_st();
-                }
-                tc_fence_before();
-                __syncwarp();
-                if (ok && lane == 0)
-                    mbar_arrive(&S.a_full);
-                cur_c = t.c;
-                ++ci;
+                bulk_commit();
+                bulk_wait_read<0>();
             }
+            __syncwarp();
+            if (ok && lane == 0)
+                mbar_arrive(&S.out_empty[os]);
+        }
+        bulk_wait<0>();
+    } else if (warp < 3 + kTransformWarps) {
+        // ------------------------------------------------------ transform
+        const int tt = threadIdx.x - 3 * 32;
+        for (int seq = 0; seq < n_it; ++seq) {
+            const BandTile t = tile_of(P, it0 + seq);
             const int s = seq % R, bs = seq & 1;
             bool ok = !*abort;
             ok = ok && mbar_wait(&S.raw_full[s], (seq / R) & 1, abort, P.budget, P.status);
@@ -371,9 +384,10 @@ __global__ void __launch_bounds__(kThreads, 1) wbmm_tc_fwd_kernel(const TcFwdPar
             ok = __all_sync(0xffffffffu, ok);
             if (ok) {
                 const uint16_t* raw =
-                    reinterpret_cast<const uint16_t*>(raw_base + (size_t)s * Cfg::RAW_BYTES);
-                transform_tile<WS>(raw, b_base + (size_t)bs * Cfg::B_BYTES, t.nb * P.nw, woff, P.W,
-                                   tw, lane);
+                    reinterpret_cast<const uint16_t*>(raw_base + (size_t)s * F::RAW_BYTES);
+                const int nwin = t.nb * P.nw;
+                transform_rows<WS>(raw, b_base + (size_t)bs * F::B_BYTES, F::SBO_B, nwin, nwin,
+                                   woff, P.W, tt, kTransformWarps * 32);
                 fence_proxy_async_smem();
             }
             __syncwarp();
@@ -382,64 +396,114 @@ __global__ void __launch_bounds__(kThreads, 1) wbmm_tc_fwd_kernel(const TcFwdPar
                 mbar_arrive(&S.raw_empty[s]);
             }
         }
+    } else if (warp < kEpiWarp0) {
+        // ------------------------------------------------------ A builders
+        const int quarter = warp & 3;
+        const int at = threadIdx.x - kBuildWarp0 * 32;  // 0..127
+        int cur_c = -1, ci = 0;
+        for (int seq = 0; seq < n_it; ++seq) {
+            const BandTile t = tile_of(P, it0 + seq);
+            if (t.c == cur_c)
+                continue;
+            bool ok = !*abort;
+            if (ci > 0)
+                ok = ok && mbar_wait(&S.a_empty, (ci - 1) & 1, abort, P.budget, P.status);
+            ok = __all_sync(0xffffffffu, ok);
+            tc_fence_after();
+            const uint16_t* Mc = nullptr;
+            if (MODE == kCached) {
+                Mc = P.src + (long long)t.c * F::D * F::D;
+            } else {
+                named_bar_sync(1, 128);   // previous channel's slices all read
+                load_tables<WS, MODE>(tc0, tc1, P.src + (long long)t.c * F::TSZ, at, 128);
+                named_bar_sync(1, 128);
+            }
+            if (ok) {
+                build_a<WS, MODE>(tmem, tc0, tc1, Mc, quarter, lane);
+                tmem_wait_st();
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (ok && lane == 0)
+                mbar_arrive(&S.a_full);
+            cur_c = t.c;
+            ++ci;
+        }
     } else {
         // ------------------------------------------------------ epilogue
+        // Eight warps: two per TMEM lane quarter.  Each takes every other
+        // 32-window chunk of the tile, loads that chunk of both M tiles with
+        // one wait, and writes bf16 outputs into the band-layout slot.
         const int quarter = warp & 3;
-        const int et = threadIdx.x - 6 * 32;  // 0..127
+        const int half = (warp - kEpiWarp0) >> 2;
+        constexpr int NCH = F::NT / 32;
         for (int seq = 0; seq < n_it; ++seq) {
-            const TileRef t = tile_ref(P, it0 + seq);
+            const BandTile t = tile_of(P, it0 + seq);
             const int nwin = t.nb * P.nw;
             const int ab = seq & 1, os = seq & 1;
             bool ok = !*abort;
             ok = ok && mbar_wait(&S.acc_full[ab], (seq >> 1) & 1, abort, P.budget, P.status);
+            if (seq >= 2)
+                ok = ok && mbar_wait(&S.out_empty[os], ((seq >> 1) - 1) & 1, abort, P.budget,
+                                     P.status);
             ok = __all_sync(0xffffffffu, ok);
             tc_fence_after();
-            if (et == 0)
-                bulk_wait_read<1>();
-            named_bar_sync(2, 128);
-            uint16_t* out = reinterpret_cast<uint16_t*>(out_base + (size_t)os * Cfg::RAW_BYTES);
+            uint16_t* out = reinterpret_cast<uint16_t*>(out_base + (size_t)os * F::RAW_BYTES);
             if (ok) {
+                const uint32_t lrow = tmem + ((uint32_t)(quarter * 32) << 16) + F::D_COL0 +
+                                      (uint32_t)(ab * F::MT * F::NT);
 #pragma unroll 1
-                for (int mt = 0; mt < Cfg::MT; ++mt) {
-                    const int u = mt * 128 + quarter * 32 + lane;
-                    const int pos = (u / WS) * P.W + (u - (u / WS) * WS);
-                    const uint32_t dcol =
-                        tmem + ((uint32_t)(quarter * 32) << 16) + Cfg::D_COL0 +
-                        (uint32_t)(ab * Cfg::MT * Cfg::NT + mt * Cfg::NT);
-#pragma unroll 1
-                    for (int c0 = 0; c0 < Cfg::NT; c0 += 32) {
-                        if (c0 >= nwin)
-                            break;
-                        uint32_t r[32];
-                        tmem_ld32(dcol + (uint32_t)c0, r);
-                        tmem_wait_ld(r);
-                        if (u < Cfg::D) {
+                for (int ch = half; ch < NCH; ch += 2) {
+                    const int c0 = ch * 32;
+                    if (c0 >= nwin)
+                        break;
+                    uint32_t r[F::MT][32];
 #pragma unroll
-                            for (int jj = 0; jj < 32; ++jj) {
-                                const int n = c0 + jj;
-                                if (n < nwin)
-                                    out[woff[n] + pos] = __bfloat16_as_ushort(
-                                        __float2bfloat16_rn(__uint_as_float(r[jj])));
-                            }
+                    for (int mt = 0; mt < F::MT; ++mt)
+                        tmem_ld32(lrow + (uint32_t)(mt * F::NT + c0), r[mt]);
+#pragma unroll
+                    for (int mt = 0; mt < F::MT; ++mt)
+                        tmem_wait_ld(r[mt]);
+                    int pos[F::MT];
+                    bool uval[F::MT];
+#pragma unroll
+                    for (int mt = 0; mt < F::MT; ++mt) {
+                        const int u = mt * 128 + quarter * 32 + lane;
+                        uval[mt] = u < F::D;
+                        pos[mt] = (u / WS) * P.W + (u - (u / WS) * WS);
+                    }
+                    // window offsets walked in registers: band k, column j
+                    int wk = c0 / P.nw, wj = c0 - wk * P.nw;
+                    int wo = wk * WS * P.W + wj * WS;
+                    const int band_step = WS * P.W - (P.nw - 1) * WS;
+#pragma unroll
+                    for (int jj = 0; jj < 32; ++jj) {
+                        const int n = c0 + jj;
+                        if (n < nwin) {
+                            uint16_t* o = out + wo;
+#pragma unroll
+                            for (int mt = 0; mt < F::MT; ++mt)
+                                if (uval[mt])
+                                    o[pos[mt]] = __bfloat16_as_ushort(
+                                        __float2bfloat16_rn(__uint_as_float(r[mt][jj])));
+                        }
+                        if (++wj == P.nw) {
+                            wj = 0;
+                            wo += band_step;
+                        } else {
+                            wo += WS;
                         }
                     }
                 }
             }
             tc_fence_before();
-            __syncwarp();
-            if (ok && lane == 0)
-                mbar_arrive(&S.acc_empty[ab]);
             fence_proxy_async_smem();
-            named_bar_sync(2, 128);
-            if (et == 0 && ok && !*abort) {
-                for_each_run<WS>(P, t, [&](long long goff, uint32_t soff, uint32_t nbytes) {
-                    bulk_s2g(P.y + goff, reinterpret_cast<const uint8_t*>(out) + soff, nbytes);
-                });
-                bulk_commit();
+            __syncwarp();
+            if (ok && lane == 0) {
+                mbar_arrive(&S.acc_empty[ab]);
+                mbar_arrive(&S.out_full[os]);
             }
         }
-        if (et == 0)
-            bulk_wait<0>();
     }
 
     tc_fence_before();
@@ -454,44 +518,43 @@ __global__ void __launch_bounds__(kThreads, 1) wbmm_tc_fwd_kernel(const TcFwdPar
 // ------------------------------------------------------------------ host
 namespace {
 
-template <int WS>
-struct FwdLayout {
-    uint32_t off_raw, off_b, off_out, off_tbl, off_woff, off_bar, total;
-    int R;
-};
-
 constexpr uint32_t kSmemMax = 232448;
 constexpr uint32_t kMinSmem = 120 * 1024;
 
 inline uint32_t align_up(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
 
+struct FwdLayout {
+    uint32_t off_raw, off_b, off_out, off_tbl, off_woff, off_bar, total;
+    int R;
+};
+
 template <int WS>
-FwdLayout<WS> fwd_layout()
+FwdLayout fwd_layout()
 {
-    using Cfg = FwdCfg<WS>;
-    FwdLayout<WS> L;
-    const uint32_t fixed = 2 * Cfg::B_BYTES + 2 * Cfg::RAW_BYTES + 4 * Cfg::TBL_BYTES +
-                           Cfg::NT * 4 + align_up(sizeof(Bars), 16) + 3 * 1024;
-    int R = (int)((kSmemMax - fixed) / Cfg::RAW_BYTES);
+    using F = FwdCfg<WS>;
+    FwdLayout L;
+    const uint32_t fixed = 2 * F::B_BYTES + 2 * F::RAW_BYTES + 2 * F::TCOPY_BYTES + F::NT * 4 +
+                           align_up(sizeof(Bars), 16) + 3 * 1024;
+    int R = (int)((kSmemMax - fixed) / F::RAW_BYTES);
     if (R > kMaxRing)
         R = kMaxRing;
     L.R = R;
     uint32_t off = 0;
     L.off_b = off;                       // operand stages first: 1024-aligned
-    off += 2 * Cfg::B_BYTES;
+    off += 2 * F::B_BYTES;
     L.off_raw = align_up(off, 128);
-    off = L.off_raw + (uint32_t)R * Cfg::RAW_BYTES;
+    off = L.off_raw + (uint32_t)R * F::RAW_BYTES;
     L.off_out = align_up(off, 128);
-    off = L.off_out + 2 * Cfg::RAW_BYTES;
+    off = L.off_out + 2 * F::RAW_BYTES;
     L.off_tbl = align_up(off, 16);
-    off = L.off_tbl + 4 * Cfg::TBL_BYTES;
+    off = L.off_tbl + 2 * F::TCOPY_BYTES;
     L.off_woff = align_up(off, 16);
-    off = L.off_woff + Cfg::NT * 4;
+    off = L.off_woff + F::NT * 4;
     L.off_bar = align_up(off, 16);
     off = L.off_bar + sizeof(Bars);
     L.total = align_up(off, 1024);
-    // at least half the SM's shared memory: one CTA (and one 512-column
-    // TMEM allocation) per SM
+    // at least half the SM's shared memory: one CTA (and one 512-column TMEM
+    // allocation) per SM
     if (L.total < kMinSmem)
         L.total = kMinSmem;
     return L;
@@ -500,8 +563,8 @@ FwdLayout<WS> fwd_layout()
 template <int WS, int MODE>
 cudaError_t launch_ws(const Geom& g, const void* x, const void* src, void* y, const Launch& L)
 {
-    using Cfg = FwdCfg<WS>;
-    const FwdLayout<WS> lay = fwd_layout<WS>();
+    using F = FwdCfg<WS>;
+    const FwdLayout lay = fwd_layout<WS>();
     if (lay.R < 2 || lay.total > kSmemMax)
         return cudaErrorInvalidConfiguration;
     static unsigned long long configured = 0;
@@ -520,21 +583,30 @@ cudaError_t launch_ws(const Geom& g, const void* x, const void* src, void* y, co
     P.src = static_cast<const uint16_t*>(src);
     P.y = static_cast<uint16_t*>(y);
     P.C = g.C; P.H = g.H; P.W = g.W; P.nh = g.nh; P.nw = g.nw;
-    P.bpt = Cfg::NT / g.nw;
-    P.bands = g.bands;
-    P.tpc = (int)((g.bands + P.bpt - 1) / P.bpt);
-    P.items = (long long)g.C * P.tpc;
+    P.bpt = F::NT / g.nw;
+    P.bands = (int)g.bands;
+    P.tpc = (P.bands + P.bpt - 1) / P.bpt;
+    P.items = g.C * P.tpc;
     P.R = lay.R;
+    P.use_tmap = 0;
+    P.kimg = 0;
+    if (P.bpt % g.nh == 0) {
+        const int k = P.bpt / g.nh;
+        if (encode_plane_map(&P.map_x, x, g, k) && encode_plane_map(&P.map_y, y, g, k)) {
+            P.use_tmap = 1;
+            P.kimg = k;
+        }
+    }
     P.off_raw = lay.off_raw; P.off_b = lay.off_b; P.off_out = lay.off_out;
     P.off_tbl = lay.off_tbl; P.off_woff = lay.off_woff; P.off_bar = lay.off_bar;
     P.budget = L.budget;
     P.status = L.status;
-    long long grid = L.num_sms;
+    int grid = L.num_sms;
     if (grid > P.items)
         grid = P.items;
     if (grid < 1)
         return cudaSuccess;
-    wbmm_tc_fwd_kernel<WS, MODE><<<(unsigned)grid, kThreads, lay.total, L.stream>>>(P);
+    wbmm_tc_fwd_kernel<WS, MODE><<<grid, kThreads, lay.total, L.stream>>>(P);
     note_launches(1);
     return cudaGetLastError();
 }
@@ -568,6 +640,9 @@ bool tc_fwd_supported(const Geom& g, bool fused)
         return false;
     // bulk copies move whole bands: 16-byte multiples
     if (((long long)g.w * g.W * 2) % 16 != 0)
+        return false;
+    // 32-bit tile bookkeeping
+    if (g.bands * (long long)g.C >= (1ll << 31))
         return false;
     return true;
 }
