@@ -30,6 +30,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 import synth  # noqa: E402
+from windowed_matmul_conv_b200.sharding import channel_range  # noqa: E402
 
 METRIC = "WBMM fwd/bwd TFLOP/s, HBM GB/s and % of roofline at w=14 bf16 on 1 B200"
 L2_BYTES = 126 * 2 ** 20
@@ -399,6 +400,7 @@ def run_gpu(args, rank, world, local_rank):
                                                        "cached_dw": "cached forward + 3x3"}[wl.kind]),
             "B": wl.B, "C_per_gpu": wl.C, "H": wl.H, "W": wl.W, "w": wl.w,
             "parallelism": "channel-sharded, %d rank(s), no collective" % world,
+            "channels_of_rank0": list(channel_range(wl.C * world, world, 0)),
             "l2": "3 rotating input/output sets, %.0f MB per step > 126 MB L2"
                   % (step_bytes(wl) / 1e6),
             "timing": "CUDA graph replay, CUDA events, max over ranks",
