@@ -142,6 +142,25 @@ WBMM_API wbmm_status wbmm_dw3x3(const void *y, const void *K, void *z,
                        int B, int C, int H, int W, wbmm_dtype dt, void *stream);
 
 /*
+ * Table gradient for callers that cannot allocate device memory: the dT of
+ * wbmm_backward (same kernels, same bits), with the fp32 partial tables kept
+ * in a fixed 4 MiB array inside the library instead of a workspace argument.
+ * The paper has no counterpart to this entry point; it exists for hosts with a
+ * fixed device-memory budget, plugins inside frameworks that own all device
+ * allocations, and paths where cudaMalloc would synchronise the device.
+ *   x, dY [B,C,H,W] dtype dt;  dT [C,(2w-1)^2] fp32 (overwritten)
+ * Allocates nothing and frees nothing.  The first call on a device looks up
+ * the array's device address (cudaGetSymbolAddress); make that first call
+ * before any stream capture.  Every device holds the array until exit.  All
+ * calls share it, so calls whose work overlaps on the GPU race and must be
+ * ordered by the caller.  Returns WBMM_ERR_WORKSPACE when C times the number
+ * of partial tables times (2w-1)^2 exceeds 2^20 floats.
+ */
+WBMM_API wbmm_status wbmm_backward_dt_static(const void *x, const void *dY, float *dT,
+                                             int B, int C, int H, int W, int w,
+                                             wbmm_dtype dt, void *stream);
+
+/*
  * Synchronises `stream`, then reports and clears the device status word that
  * kernels set when a bounded wait expires (WBMM_ERR_TIMEOUT), or returns
  * WBMM_ERR_CUDA for a sticky CUDA error.  WBMM_OK otherwise.

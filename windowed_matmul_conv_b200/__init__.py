@@ -35,7 +35,8 @@ STATUS_NAMES = {0: "WBMM_OK", 1: "WBMM_ERR_INVALID_ARG", 2: "WBMM_ERR_SHAPE",
 EXPORTS = ("wbmm_forward", "wbmm_backward_workspace_bytes", "wbmm_backward",
            "wbmm_cache_matrices", "wbmm_forward_cached", "wbmm_dw3x3",
            "wbmm_get_device_status", "wbmm_status_string", "wbmm_set_wait_budget",
-           "wbmm_wait_selftest", "wbmm_launch_count", "wbmm_last_path")
+           "wbmm_wait_selftest", "wbmm_launch_count", "wbmm_last_path",
+           "wbmm_backward_dt_static")
 
 _vp, _i, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
 _lib.wbmm_forward.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]
@@ -43,6 +44,7 @@ _lib.wbmm_backward_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, _i]
 _lib.wbmm_backward_workspace_bytes.restype = _sz
 _lib.wbmm_backward.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _sz, _i, _i, _i, _i, _i, _i, _vp]
 _lib.wbmm_cache_matrices.argtypes = [_vp, _vp, _i, _i, _i, _vp]
+_lib.wbmm_backward_dt_static.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]
 _lib.wbmm_forward_cached.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]
 _lib.wbmm_dw3x3.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]
 _lib.wbmm_get_device_status.argtypes = [_vp]
@@ -54,7 +56,8 @@ _lib.wbmm_wait_selftest.argtypes = [ctypes.c_ulonglong, _vp]
 _lib.wbmm_launch_count.argtypes = []
 _lib.wbmm_launch_count.restype = ctypes.c_ulonglong
 _lib.wbmm_last_path.argtypes = []
-for _f in ("wbmm_forward", "wbmm_backward", "wbmm_cache_matrices", "wbmm_forward_cached",
+for _f in ("wbmm_forward", "wbmm_backward", "wbmm_backward_dt_static", "wbmm_cache_matrices",
+           "wbmm_forward_cached",
            "wbmm_dw3x3", "wbmm_get_device_status", "wbmm_wait_selftest", "wbmm_last_path"):
     getattr(_lib, _f).restype = _i
 
@@ -114,6 +117,13 @@ def wbmm_backward(x, T, dY, dX, dT, workspace, w, stream=None):
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(_lib.wbmm_backward(_p(x), _p(T), _p(dY), _p(dX), _p(dT), _p(workspace), ws_bytes,
                               B, C, H, W, int(w), _dt(dY), _stream(stream)))
+
+
+def wbmm_backward_dt_static(x, dY, dT, w, stream=None):
+    """dT of wbmm_backward with the library's fixed scratch array (no allocation)."""
+    B, C, H, W = _map_shape(dY)
+    _check(_lib.wbmm_backward_dt_static(_p(x), _p(dY), _p(dT), B, C, H, W, int(w), _dt(dY),
+                                        _stream(stream)))
 
 
 def wbmm_cache_matrices(T, M, w, stream=None):

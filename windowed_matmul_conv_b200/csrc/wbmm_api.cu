@@ -131,6 +131,8 @@ int dt_chunks_for(const Geom& g, wbmm_dtype dt)
 
 void note_launches(int n) { g_launches.fetch_add((unsigned long long)n); }
 
+int launch_for_stream(void* stream, Launch* L) { return (int)make_launch(stream, L); }
+
 }  // namespace wbmm
 
 using namespace wbmm;

@@ -79,4 +79,8 @@ cudaError_t wait_selftest_launch(unsigned long long cycles, const Launch& L);
 
 void note_launches(int n);
 
+// Launch settings (stream, SM count, status word, wait budget) for the
+// current device; returns a wbmm_status code (0 on success).
+int launch_for_stream(void* stream, Launch* L);
+
 }  // namespace wbmm
