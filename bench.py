@@ -242,6 +242,22 @@ def prefill(ms=20.0):
     torch.cuda._sleep(int(ms * 1e6 * 2.0))   # ~2 GHz cycles per ns
 
 
+def recorded_traffic(kernel):
+    """DRAM bytes per launch from the committed ncu capture, or None when the
+    kernel source changed since the counters were taken."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            rec = json.load(f).get(kernel)
+        if not rec:
+            return None
+        with open(os.path.join(ROOT, rec["source"]), "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()[:16]
+        return rec["bytes"] if sha == rec["sha256_16"] else None
+    except (OSError, ValueError, KeyError):
+        return None
+
+
 def cpu_baseline(wl, host, budget_s=10.0):
     """The oracle, as it stands, on a bounded sample: the first images of the
     same inputs (all channels), repeated until `budget_s` of CPU time."""
@@ -419,7 +435,8 @@ def run_gpu(args, rank, world, local_rank):
         result["roofline"] = {"bound": "hbm", "kernel": dom, "achieved": kern[dom]["gbs"],
                               "peak": peaks["hbm_gbs"], "unit": "GB/s",
                               "frac": round(kern[dom]["gbs"] / peaks["hbm_gbs"], 4),
-                              "traffic": None, "peak_source": peaks["source"]}
+                              "traffic": recorded_traffic(dom) if wl.name == "train_bf16" else None,
+                              "peak_source": peaks["source"]}
     else:
         result["roofline"] = {"bound": "tensor", "kernel": dom, "achieved": kern[dom]["tflops"],
                               "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",

@@ -151,8 +151,9 @@ def test_forward_cached_bf16(shape):
 
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
-def test_dw3x3(dtype):
-    y = gen((3, 4, 37, 70), 16, dtype)
+@pytest.mark.parametrize("hw", [(37, 70), (40, 64), (33, 8)])  # scalar and 16-byte-row paths
+def test_dw3x3(dtype, hw):
+    y = gen((3, 4) + hw, 16, dtype)
     K = gen((4, 1, 3, 3), 17, dtype, 1.0 / 3.0)
     z = wb.dw3x3(y, K)
     torch.cuda.synchronize()

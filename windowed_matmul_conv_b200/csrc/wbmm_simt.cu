@@ -197,6 +197,77 @@ __global__ void dw3x3_kernel(const TIn* __restrict__ y, const TIn* __restrict__ 
     }
 }
 
+// bf16 maps whose rows are whole 16-byte vectors (W % 8 == 0): a band of
+// kDwVecRows output rows plus one halo row above and below is staged in
+// shared memory with 16-byte loads; each thread makes 8 consecutive outputs
+// and writes them as one 16-byte store.  Same fp32 fused multiply-add order
+// as dw3x3_kernel (a outer, e inner, zero padding included), so both kernels
+// give the same bits.
+constexpr int kDwVecRows = 16;
+
+__global__ void __launch_bounds__(256) dw3x3_bf16_vec_kernel(const uint16_t* __restrict__ y,
+                                                             const uint16_t* __restrict__ K,
+                                                             uint16_t* __restrict__ z, int C,
+                                                             int H, int W, int tiles_y)
+{
+    extern __shared__ uint4 sband[];
+    const int nvec = W / 8;
+    const long long bc = blockIdx.x / tiles_y;
+    const int ty = blockIdx.x - (int)(bc * tiles_y);
+    const int c = (int)(bc % C);
+    const int h0 = ty * kDwVecRows;
+    const uint4* yp = reinterpret_cast<const uint4*>(y) + bc * H * (long long)nvec;
+    for (int e = threadIdx.x; e < (kDwVecRows + 2) * nvec; e += blockDim.x) {
+        const int rr = e / nvec, v = e - (e / nvec) * nvec;
+        const int h = h0 - 1 + rr;
+        sband[e] = (h >= 0 && h < H) ? __ldg(yp + (long long)h * nvec + v) : make_uint4(0, 0, 0, 0);
+    }
+    float k[9];
+#pragma unroll
+    for (int m = 0; m < 9; ++m)
+        k[m] = __bfloat162float(__ushort_as_bfloat16(K[c * 9 + m]));
+    __syncthreads();
+    const uint16_t* s16 = reinterpret_cast<const uint16_t*>(sband);
+    uint4* zp = reinterpret_cast<uint4*>(z) + bc * H * (long long)nvec;
+    for (int o = threadIdx.x; o < kDwVecRows * nvec; o += blockDim.x) {
+        const int rr = o / nvec, v = o - (o / nvec) * nvec;
+        const int h = h0 + rr;
+        if (h >= H)
+            continue;
+        float acc[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            acc[j] = 0.0f;
+#pragma unroll
+        for (int a = 0; a < 3; ++a) {
+            const uint16_t* row = s16 + (long long)(rr + a) * W + 8 * v;
+            float vals[10];
+            vals[0] = v > 0 ? __bfloat162float(__ushort_as_bfloat16(row[-1])) : 0.0f;
+            const uint4 mid = sband[(rr + a) * nvec + v];
+            const uint32_t w4[4] = {mid.x, mid.y, mid.z, mid.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                vals[1 + 2 * j] = __uint_as_float(w4[j] << 16);
+                vals[2 + 2 * j] = __uint_as_float(w4[j] & 0xFFFF0000u);
+            }
+            vals[9] = v + 1 < nvec ? __bfloat162float(__ushort_as_bfloat16(row[8])) : 0.0f;
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+#pragma unroll
+                for (int e = 0; e < 3; ++e)
+                    acc[j] = __fmaf_rn(k[a * 3 + e], vals[j + e], acc[j]);
+        }
+        uint32_t packed[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t lo = __bfloat16_as_ushort(__float2bfloat16_rn(acc[2 * j]));
+            const uint32_t hi = __bfloat16_as_ushort(__float2bfloat16_rn(acc[2 * j + 1]));
+            packed[j] = lo | (hi << 16);
+        }
+        zp[(long long)h * nvec + v] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+    }
+}
+
 // ------------------------------------------------ bounded-wait self-test
 __global__ void wait_selftest_kernel(unsigned long long cycles, int* status)
 {
@@ -328,6 +399,22 @@ cudaError_t cache_matrices_launch(int C, int w, bool is_bf16, const void* T, voi
 cudaError_t dw3x3_launch(const Geom& g, bool is_bf16, const void* y, const void* K, void* z,
                          const Launch& L)
 {
+    if (is_bf16 && g.W % 8 == 0 && reinterpret_cast<uintptr_t>(y) % 16 == 0 &&
+        reinterpret_cast<uintptr_t>(z) % 16 == 0) {
+        const int ty = (g.H + kDwVecRows - 1) / kDwVecRows;
+        const long long blocks = (long long)g.B * g.C * ty;
+        const size_t smem = (size_t)(kDwVecRows + 2) * (g.W / 8) * 16;
+        if (blocks > 0 && blocks <= 0x7fffffffLL && smem <= kSimtSmemMax) {
+            cudaError_t e = set_smem(dw3x3_bf16_vec_kernel, smem);
+            if (e != cudaSuccess)
+                return e;
+            dw3x3_bf16_vec_kernel<<<(unsigned)blocks, 256, smem, L.stream>>>(
+                static_cast<const uint16_t*>(y), static_cast<const uint16_t*>(K),
+                static_cast<uint16_t*>(z), g.C, g.H, g.W, ty);
+            note_launches(1);
+            return cudaGetLastError();
+        }
+    }
     const int ty = (g.H + kDwTH - 1) / kDwTH, tx = (g.W + kDwTW - 1) / kDwTW;
     const long long blocks = (long long)g.B * g.C * ty * tx;
     if (blocks == 0)
