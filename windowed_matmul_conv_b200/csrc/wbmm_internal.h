@@ -5,6 +5,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <utility>
 
 namespace wbmm {
 
@@ -78,6 +79,26 @@ cudaError_t dw3x3_launch(const Geom& g, bool is_bf16, const void* y, const void*
 cudaError_t wait_selftest_launch(unsigned long long cycles, const Launch& L);
 
 void note_launches(int n);
+
+// Launches `kernel` with programmatic stream serialization: it may begin its
+// prologue while the previous kernel in the stream drains, and every library
+// kernel calls grid_dep_wait() before reading or writing tensors.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args&&... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // Launch settings (stream, SM count, status word, wait budget) for the
 // current device; returns a wbmm_status code (0 on success).

@@ -32,6 +32,8 @@ __global__ void simt_fwd_kernel(const TIn* __restrict__ x, const TIn* __restrict
 {
     extern __shared__ float sm[];
     const int tsz = (2 * w - 1) * (2 * w - 1), d = w * w;
+    grid_dep_wait();
+    grid_dep_launch();
     const long long blk = blockIdx.x;
     const long long bc = blk / nh;
     const int i = (int)(blk - bc * nh);
@@ -82,6 +84,8 @@ __global__ void simt_dt_kernel(const TIn* __restrict__ x, const TIn* __restrict_
                                int nw, long long bands, int chunks)
 {
     extern __shared__ float sm[];
+    grid_dep_wait();
+    grid_dep_launch();
     const int tsz = (2 * w - 1) * (2 * w - 1);
     const int c = blockIdx.x / chunks, k = blockIdx.x - (blockIdx.x / chunks) * chunks;
     float* xb = sm;
@@ -128,6 +132,8 @@ __global__ void simt_dt_kernel(const TIn* __restrict__ x, const TIn* __restrict_
 __global__ void dt_finalize_kernel(const float* __restrict__ part, float* __restrict__ dT, int C,
                                    int tsz, int chunks)
 {
+    grid_dep_wait();
+    grid_dep_launch();
     const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= (long long)C * tsz)
         return;
@@ -142,6 +148,8 @@ __global__ void dt_finalize_kernel(const float* __restrict__ part, float* __rest
 template <typename E>
 __global__ void cache_kernel(const E* __restrict__ T, E* __restrict__ M, int C, int w)
 {
+    grid_dep_wait();
+    grid_dep_launch();
     const int d = w * w, tsz = (2 * w - 1) * (2 * w - 1);
     const long long total = (long long)C * d * d;
     for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < total;
@@ -163,6 +171,8 @@ template <typename TIn>
 __global__ void dw3x3_kernel(const TIn* __restrict__ y, const TIn* __restrict__ K,
                              TIn* __restrict__ z, int C, int H, int W, int tiles_y, int tiles_x)
 {
+    grid_dep_wait();
+    grid_dep_launch();
     __shared__ float tile[(kDwTH + 2) * (kDwTW + 2)];
     const long long blk = blockIdx.x;
     const long long bc = blk / ((long long)tiles_y * tiles_x);
@@ -210,6 +220,8 @@ __global__ void __launch_bounds__(256) dw3x3_bf16_vec_kernel(const uint16_t* __r
                                                              uint16_t* __restrict__ z, int C,
                                                              int H, int W, int tiles_y)
 {
+    grid_dep_wait();
+    grid_dep_launch();
     extern __shared__ uint4 sband[];
     const int nvec = W / 8;
     const long long bc = blockIdx.x / tiles_y;
@@ -271,6 +283,8 @@ __global__ void __launch_bounds__(256) dw3x3_bf16_vec_kernel(const uint16_t* __r
 // ------------------------------------------------ bounded-wait self-test
 __global__ void wait_selftest_kernel(unsigned long long cycles, int* status)
 {
+    grid_dep_wait();
+    grid_dep_launch();
     __shared__ uint64_t bar;
     __shared__ int abort_flag;
     if (threadIdx.x == 0) {
@@ -315,22 +329,24 @@ cudaError_t simt_fwd_launch(const Geom& g, AMode mode, bool is_bf16, const void*
         return cudaSuccess;
     if (blocks > 0x7fffffffLL)
         return cudaErrorInvalidConfiguration;
+    const dim3 grid((unsigned)blocks), block(256);
     cudaError_t e;
     if (is_bf16) {
-        e = set_smem(simt_fwd_kernel<__nv_bfloat16>, smem);
-        if (e != cudaSuccess)
-            return e;
-        simt_fwd_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, smem, L.stream>>>(
-            static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(src),
-            static_cast<__nv_bfloat16*>(y), g.C, g.H, g.W, g.w, g.nh, g.nw, (int)mode);
+        using E = __nv_bfloat16;
+        e = set_smem(simt_fwd_kernel<E>, smem);
+        if (e == cudaSuccess)
+            e = launch_pdl(simt_fwd_kernel<E>, grid, block, smem, L.stream,
+                           static_cast<const E*>(x), static_cast<const E*>(src),
+                           static_cast<E*>(y), g.C, g.H, g.W, g.w, g.nh, g.nw, (int)mode);
     } else {
         e = set_smem(simt_fwd_kernel<float>, smem);
-        if (e != cudaSuccess)
-            return e;
-        simt_fwd_kernel<float><<<(unsigned)blocks, 256, smem, L.stream>>>(
-            static_cast<const float*>(x), static_cast<const float*>(src), static_cast<float*>(y),
-            g.C, g.H, g.W, g.w, g.nh, g.nw, (int)mode);
+        if (e == cudaSuccess)
+            e = launch_pdl(simt_fwd_kernel<float>, grid, block, smem, L.stream,
+                           static_cast<const float*>(x), static_cast<const float*>(src),
+                           static_cast<float*>(y), g.C, g.H, g.W, g.w, g.nh, g.nw, (int)mode);
     }
+    if (e != cudaSuccess)
+        return e;
     note_launches(1);
     return cudaGetLastError();
 }
@@ -345,22 +361,24 @@ cudaError_t simt_dt_launch(const Geom& g, bool is_bf16, const void* x, const voi
     const long long blocks = (long long)g.C * chunks;
     if (blocks == 0)
         return cudaSuccess;
+    const dim3 grid((unsigned)blocks), block(256);
     cudaError_t e;
     if (is_bf16) {
-        e = set_smem(simt_dt_kernel<__nv_bfloat16>, smem);
-        if (e != cudaSuccess)
-            return e;
-        simt_dt_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, smem, L.stream>>>(
-            static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(dy),
-            partials, g.C, g.H, g.W, g.w, g.nh, g.nw, g.bands, chunks);
+        using E = __nv_bfloat16;
+        e = set_smem(simt_dt_kernel<E>, smem);
+        if (e == cudaSuccess)
+            e = launch_pdl(simt_dt_kernel<E>, grid, block, smem, L.stream,
+                           static_cast<const E*>(x), static_cast<const E*>(dy), partials, g.C,
+                           g.H, g.W, g.w, g.nh, g.nw, g.bands, chunks);
     } else {
         e = set_smem(simt_dt_kernel<float>, smem);
-        if (e != cudaSuccess)
-            return e;
-        simt_dt_kernel<float><<<(unsigned)blocks, 256, smem, L.stream>>>(
-            static_cast<const float*>(x), static_cast<const float*>(dy), partials, g.C, g.H, g.W,
-            g.w, g.nh, g.nw, g.bands, chunks);
+        if (e == cudaSuccess)
+            e = launch_pdl(simt_dt_kernel<float>, grid, block, smem, L.stream,
+                           static_cast<const float*>(x), static_cast<const float*>(dy), partials,
+                           g.C, g.H, g.W, g.w, g.nh, g.nw, g.bands, chunks);
     }
+    if (e != cudaSuccess)
+        return e;
     note_launches(1);
     return cudaGetLastError();
 }
@@ -371,8 +389,10 @@ cudaError_t dt_finalize_launch(int C, int tsz, int chunks, const float* partials
     const long long n = (long long)C * tsz;
     if (n == 0)
         return cudaSuccess;
-    dt_finalize_kernel<<<(unsigned)((n + 255) / 256), 256, 0, L.stream>>>(partials, dT, C, tsz,
-                                                                         chunks);
+    cudaError_t e = launch_pdl(dt_finalize_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256),
+                               0, L.stream, partials, dT, C, tsz, chunks);
+    if (e != cudaSuccess)
+        return e;
     note_launches(1);
     return cudaGetLastError();
 }
@@ -386,12 +406,16 @@ cudaError_t cache_matrices_launch(int C, int w, bool is_bf16, const void* T, voi
         blocks = (long long)L.num_sms * 32;
     if (blocks < 1)
         return cudaSuccess;
+    const dim3 grid((unsigned)blocks), block(256);
+    cudaError_t e;
     if (is_bf16)
-        cache_kernel<uint16_t><<<(unsigned)blocks, 256, 0, L.stream>>>(
-            static_cast<const uint16_t*>(T), static_cast<uint16_t*>(M), C, w);
+        e = launch_pdl(cache_kernel<uint16_t>, grid, block, 0, L.stream,
+                       static_cast<const uint16_t*>(T), static_cast<uint16_t*>(M), C, w);
     else
-        cache_kernel<uint32_t><<<(unsigned)blocks, 256, 0, L.stream>>>(
-            static_cast<const uint32_t*>(T), static_cast<uint32_t*>(M), C, w);
+        e = launch_pdl(cache_kernel<uint32_t>, grid, block, 0, L.stream,
+                       static_cast<const uint32_t*>(T), static_cast<uint32_t*>(M), C, w);
+    if (e != cudaSuccess)
+        return e;
     note_launches(1);
     return cudaGetLastError();
 }
@@ -406,11 +430,13 @@ cudaError_t dw3x3_launch(const Geom& g, bool is_bf16, const void* y, const void*
         const size_t smem = (size_t)(kDwVecRows + 2) * (g.W / 8) * 16;
         if (blocks > 0 && blocks <= 0x7fffffffLL && smem <= kSimtSmemMax) {
             cudaError_t e = set_smem(dw3x3_bf16_vec_kernel, smem);
+            if (e == cudaSuccess)
+                e = launch_pdl(dw3x3_bf16_vec_kernel, dim3((unsigned)blocks), dim3(256), smem,
+                               L.stream, static_cast<const uint16_t*>(y),
+                               static_cast<const uint16_t*>(K), static_cast<uint16_t*>(z), g.C,
+                               g.H, g.W, ty);
             if (e != cudaSuccess)
                 return e;
-            dw3x3_bf16_vec_kernel<<<(unsigned)blocks, 256, smem, L.stream>>>(
-                static_cast<const uint16_t*>(y), static_cast<const uint16_t*>(K),
-                static_cast<uint16_t*>(z), g.C, g.H, g.W, ty);
             note_launches(1);
             return cudaGetLastError();
         }
@@ -421,21 +447,29 @@ cudaError_t dw3x3_launch(const Geom& g, bool is_bf16, const void* y, const void*
         return cudaSuccess;
     if (blocks > 0x7fffffffLL)
         return cudaErrorInvalidConfiguration;
-    if (is_bf16)
-        dw3x3_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, L.stream>>>(
-            static_cast<const __nv_bfloat16*>(y), static_cast<const __nv_bfloat16*>(K),
-            static_cast<__nv_bfloat16*>(z), g.C, g.H, g.W, ty, tx);
-    else
-        dw3x3_kernel<float><<<(unsigned)blocks, 256, 0, L.stream>>>(
-            static_cast<const float*>(y), static_cast<const float*>(K), static_cast<float*>(z),
-            g.C, g.H, g.W, ty, tx);
+    const dim3 grid((unsigned)blocks), block(256);
+    cudaError_t e;
+    if (is_bf16) {
+        using E = __nv_bfloat16;
+        e = launch_pdl(dw3x3_kernel<E>, grid, block, 0, L.stream, static_cast<const E*>(y),
+                       static_cast<const E*>(K), static_cast<E*>(z), g.C, g.H, g.W, ty, tx);
+    } else {
+        e = launch_pdl(dw3x3_kernel<float>, grid, block, 0, L.stream,
+                       static_cast<const float*>(y), static_cast<const float*>(K),
+                       static_cast<float*>(z), g.C, g.H, g.W, ty, tx);
+    }
+    if (e != cudaSuccess)
+        return e;
     note_launches(1);
     return cudaGetLastError();
 }
 
 cudaError_t wait_selftest_launch(unsigned long long cycles, const Launch& L)
 {
-    wait_selftest_kernel<<<1, 32, 0, L.stream>>>(cycles, L.status);
+    cudaError_t e = launch_pdl(wait_selftest_kernel, dim3(1), dim3(32), 0, L.stream, cycles,
+                               L.status);
+    if (e != cudaSuccess)
+        return e;
     note_launches(1);
     return cudaGetLastError();
 }

@@ -186,6 +186,10 @@ __global__ void __launch_bounds__(kDtThreads, 1) wbmm_tc_dt_kernel(const __grid_
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = S.tmem_slot;
+    // Everything above overlaps the previous kernel's tail; tensors are read
+    // and written only after it has completed.
+    grid_dep_wait();
+    grid_dep_launch();
 
     if (warp == 0) {
         // ------------------------------------------------------ producer
@@ -523,7 +527,10 @@ cudaError_t dt_launch_ws(const Geom& g, const void* x, const void* dy, float* pa
         grid = P.items;
     if (grid < 1)
         return cudaSuccess;
-    wbmm_tc_dt_kernel<WS><<<grid, kDtThreads, lay.total, L.stream>>>(P);
+    cudaError_t e = launch_pdl(wbmm_tc_dt_kernel<WS>, dim3(grid), dim3(kDtThreads), lay.total,
+                               L.stream, P);
+    if (e != cudaSuccess)
+        return e;
     note_launches(1);
     return cudaGetLastError();
 }

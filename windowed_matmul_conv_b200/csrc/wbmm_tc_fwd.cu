@@ -92,8 +92,8 @@ struct Bars {
     uint64_t acc_empty[2];
     uint64_t out_full[2];
     uint64_t out_empty[2];
-    uint64_t a_full;
-    uint64_t a_empty;
+    uint64_t a_full[2];     // per M tile
+    uint64_t a_empty[2];
     uint64_t fin;
     uint32_t tmem_slot;
     int abort;
@@ -132,66 +132,62 @@ __device__ __forceinline__ void load_tables(uint16_t* c0, uint16_t* c1, const ui
     }
 }
 
-// Writes this warp's 32 lanes (rows u) of the A operand into TMEM: for each
-// window row r the RP/2 columns holding slots r*RP .. r*RP+RP-1.
+// Writes this warp's 32 lanes (rows u) of M tile `mt` of the A operand into
+// TMEM: for each window row r the RP/2 columns holding slots r*RP .. +RP-1.
 template <int WS, int MODE>
 __device__ __forceinline__ void build_a(uint32_t tmem, const uint16_t* c0, const uint16_t* c1,
-                                        const uint16_t* Mc, int quarter, int lane)
+                                        const uint16_t* Mc, int quarter, int lane, int mt)
 {
     using F = FwdCfg<WS>;
-#pragma unroll 1
-    for (int mt = 0; mt < F::MT; ++mt) {
-        const int u = mt * 128 + quarter * 32 + lane;
-        const bool uval = u < F::D;
-        const int p = uval ? u / WS : 0, q = uval ? u - (u / WS) * WS : 0;
-        const int col0 = WS - 1 - q;                       // first table column of a slice
-        const uint16_t* tcopy = (col0 & 1) ? c1 : c0;
-        const int cbase = col0 & ~1;
-        const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(mt * (F::KP / 2));
-#pragma unroll 1
-        for (int r = 0; r < WS; ++r) {
-            uint32_t wv[F::RP / 2];
-            if (MODE == kCached) {
-                const uint16_t* row = Mc + (long long)u * F::D + r * WS;
+    const int u = mt * 128 + quarter * 32 + lane;
+    const bool uval = u < F::D;
+    const int p = uval ? u / WS : 0, q = uval ? u - (u / WS) * WS : 0;
+    const int col0 = WS - 1 - q;                       // first table column of a slice
+    const uint16_t* tcopy = (col0 & 1) ? c1 : c0;
+    const int cbase = col0 & ~1;
+    const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(mt * (F::KP / 2));
+#pragma unroll 2
+    for (int r = 0; r < WS; ++r) {
+        uint32_t wv[F::RP / 2];
+        if (MODE == kCached) {
+            const uint16_t* row = Mc + (long long)u * F::D + r * WS;
 #pragma unroll
-                for (int m = 0; m < F::RP / 2; ++m) {
-                    uint32_t v = 0;
-                    if (uval && 2 * m < WS) {
-                        if (WS % 2 == 0) {
-                            v = __ldg(reinterpret_cast<const unsigned int*>(row) + m);
-                        } else {
-                            const uint16_t lo = row[2 * m];
-                            const uint16_t hi = (2 * m + 1 < WS) ? row[2 * m + 1] : (uint16_t)0;
-                            v = pack_bf16x2(lo, hi);
-                        }
+            for (int m = 0; m < F::RP / 2; ++m) {
+                uint32_t v = 0;
+                if (uval && 2 * m < WS) {
+                    if (WS % 2 == 0) {
+                        v = __ldg(reinterpret_cast<const unsigned int*>(row) + m);
+                    } else {
+                        const uint16_t lo = row[2 * m];
+                        const uint16_t hi = (2 * m + 1 < WS) ? row[2 * m + 1] : (uint16_t)0;
+                        v = pack_bf16x2(lo, hi);
                     }
-                    wv[m] = v;
                 }
-            } else {
-                const int a = (MODE == kTable) ? (p - r + WS - 1) : (r - p + WS - 1);
-                const uint32_t* srow =
-                    reinterpret_cast<const uint32_t*>(tcopy + a * F::TROW + cbase);
-#pragma unroll
-                for (int m = 0; m < F::RP / 2; ++m) {
-                    uint32_t v = (uval && 2 * m < WS) ? srow[m] : 0u;
-                    if (WS % 2 == 1 && 2 * m + 1 == WS)
-                        v &= 0xFFFFu;
-                    wv[m] = v;
-                }
+                wv[m] = v;
             }
-            if constexpr (F::RP == 16) {
-                tmem_st8(taddr + (uint32_t)(r * 8), wv);
-            } else {
-                tmem_st4(taddr + (uint32_t)(r * 4), wv);
+        } else {
+            const int a = (MODE == kTable) ? (p - r + WS - 1) : (r - p + WS - 1);
+            const uint32_t* srow = reinterpret_cast<const uint32_t*>(tcopy + a * F::TROW + cbase);
+#pragma unroll
+            for (int m = 0; m < F::RP / 2; ++m) {
+                uint32_t v = (uval && 2 * m < WS) ? srow[m] : 0u;
+                if (WS % 2 == 1 && 2 * m + 1 == WS)
+                    v &= 0xFFFFu;
+                wv[m] = v;
             }
         }
-        if (F::KP > F::K) {
-            // zero the K columns past the last window row (odd small w)
-            const uint32_t z[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-            for (int cc = F::K / 2; cc < F::KP / 2; cc += 4)
-                tmem_st4(taddr + (uint32_t)cc, z);
+        if constexpr (F::RP == 16) {
+            tmem_st8(taddr + (uint32_t)(r * 8), wv);
+        } else {
+            tmem_st4(taddr + (uint32_t)(r * 4), wv);
         }
+    }
+    if (F::KP > F::K) {
+        // zero the K columns past the last window row (odd small w)
+        const uint32_t z[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+        for (int cc = F::K / 2; cc < F::KP / 2; cc += 4)
+            tmem_st4(taddr + (uint32_t)cc, z);
     }
 }
 
@@ -230,8 +226,10 @@ __global__ void __launch_bounds__(kThreads, 1) wbmm_tc_fwd_kernel(const __grid_c
             mbar_init(&S.out_full[i], kEpiWarps);
             mbar_init(&S.out_empty[i], 1);
         }
-        mbar_init(&S.a_full, 4);
-        mbar_init(&S.a_empty, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&S.a_full[i], 4);
+            mbar_init(&S.a_empty[i], 1);
+        }
         mbar_init(&S.fin, 1);
         S.abort = 0;
         fence_mbar_init();
@@ -253,6 +251,10 @@ __global__ void __launch_bounds__(kThreads, 1) wbmm_tc_fwd_kernel(const __grid_c
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = S.tmem_slot;
+    // Everything above overlaps the previous kernel's tail; tensors are read
+    // and written only after it has completed.
+    grid_dep_wait();
+    grid_dep_launch();
 
     if (warp == 0) {
         // ------------------------------------------------------ producer
@@ -304,8 +306,8 @@ __global__ void __launch_bounds__(kThreads, 1) wbmm_tc_fwd_kernel(const __grid_c
             for (int seq = 0; seq < n_it; ++seq) {
                 const BandTile t = tile_of(P, it0 + seq);
                 bool ok = !*abort;
-                if (t.c != cur_c) {
-                    ok = ok && mbar_wait(&S.a_full, ci & 1, abort, P.budget, P.status);
+                const bool first_of_channel = t.c != cur_c;
+                if (first_of_channel) {
                     cur_c = t.c;
                     ++ci;
                 }
@@ -314,28 +316,34 @@ __global__ void __launch_bounds__(kThreads, 1) wbmm_tc_fwd_kernel(const __grid_c
                 if (seq >= 2)
                     ok = ok && mbar_wait(&S.acc_empty[ab], ((seq >> 1) - 1) & 1, abort, P.budget,
                                          P.status);
-                if (!ok)
-                    continue;
-                tc_fence_after();
+                const bool last_of_channel =
+                    (seq == n_it - 1) || (tile_of(P, it0 + seq + 1).c != t.c);
                 // Descriptors differ per K step only in the start-address
                 // field (+256 bytes = +16 in 16-byte units); the loop is fully
                 // unrolled so each MMA issues with a couple of integer adds.
+                // M tiles are handed over one at a time: the A builders may
+                // refill tile 0 while tile 1's last MMAs of a channel run.
                 const uint64_t bdesc0 =
                     smem_desc(smem_u32(b_base + (size_t)bs * F::B_BYTES), 128, F::SBO_B);
                 const uint32_t d0 = tmem + F::D_COL0 + (uint32_t)(ab * F::MT * F::NT);
 #pragma unroll
                 for (int mt = 0; mt < F::MT; ++mt) {
+                    if (first_of_channel)
+                        ok = ok && mbar_wait(&S.a_full[mt], (ci - 1) & 1, abort, P.budget, P.status);
+                    if (!ok)
+                        break;
+                    tc_fence_after();
 #pragma unroll
                     for (int k = 0; k < F::KSTEPS; ++k)
                         mma_ts(d0 + (uint32_t)(mt * F::NT), tmem + (uint32_t)(mt * (F::KP / 2) + k * 8),
                                bdesc0 + (uint64_t)(k * 16), F::IDESC, k > 0 ? 1u : 0u);
+                    if (last_of_channel)
+                        tc_commit(&S.a_empty[mt]);
                 }
+                if (!ok)
+                    continue;
                 tc_commit(&S.b_empty[bs]);
                 tc_commit(&S.acc_full[ab]);
-                const bool last_of_channel =
-                    (seq == n_it - 1) || (tile_of(P, it0 + seq + 1).c != t.c);
-                if (last_of_channel)
-                    tc_commit(&S.a_empty);
             }
             // Drain: all issued MMAs complete before TMEM is released.
             tc_commit(&S.fin);
@@ -405,27 +413,32 @@ __global__ void __launch_bounds__(kThreads, 1) wbmm_tc_fwd_kernel(const __grid_c
             const BandTile t = tile_of(P, it0 + seq);
             if (t.c == cur_c)
                 continue;
-            bool ok = !*abort;
-            if (ci > 0)
-                ok = ok && mbar_wait(&S.a_empty, (ci - 1) & 1, abort, P.budget, P.status);
-            ok = __all_sync(0xffffffffu, ok);
-            tc_fence_after();
             const uint16_t* Mc = nullptr;
             if (MODE == kCached) {
                 Mc = P.src + (long long)t.c * F::D * F::D;
             } else {
+                // the tables live in shared memory: they can be refilled
+                // before the previous channel's MMAs release TMEM
                 named_bar_sync(1, 128);   // previous channel's slices all read
                 load_tables<WS, MODE>(tc0, tc1, P.src + (long long)t.c * F::TSZ, at, 128);
                 named_bar_sync(1, 128);
             }
-            if (ok) {
-                build_a<WS, MODE>(tmem, tc0, tc1, Mc, quarter, lane);
-                tmem_wait_st();
+            bool ok = !*abort;
+#pragma unroll 1
+            for (int mt = 0; mt < F::MT; ++mt) {
+                if (ci > 0)
+                    ok = ok && mbar_wait(&S.a_empty[mt], (ci - 1) & 1, abort, P.budget, P.status);
+                ok = __all_sync(0xffffffffu, ok);
+                tc_fence_after();
+                if (ok) {
+                    build_a<WS, MODE>(tmem, tc0, tc1, Mc, quarter, lane, mt);
+                    tmem_wait_st();
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (ok && lane == 0)
+                    mbar_arrive(&S.a_full[mt]);
             }
-            tc_fence_before();
-            __syncwarp();
-            if (ok && lane == 0)
-                mbar_arrive(&S.a_full);
             cur_c = t.c;
             ++ci;
         }
@@ -606,7 +619,10 @@ cudaError_t launch_ws(const Geom& g, const void* x, const void* src, void* y, co
         grid = P.items;
     if (grid < 1)
         return cudaSuccess;
-    wbmm_tc_fwd_kernel<WS, MODE><<<grid, kThreads, lay.total, L.stream>>>(P);
+    cudaError_t e = launch_pdl(wbmm_tc_fwd_kernel<WS, MODE>, dim3(grid), dim3(kThreads),
+                               lay.total, L.stream, P);
+    if (e != cudaSuccess)
+        return e;
     note_launches(1);
     return cudaGetLastError();
 }
