@@ -184,6 +184,12 @@ wbmm_status wbmm_forward(const void* x, const void* T, void* y, int B, int C, in
     Launch L;
     if ((st = make_launch(stream, &L)) != WBMM_OK)
         return st;
+    if (dt == WBMM_BF16 && tc_toep_supported(g)) {
+        st = from_cuda(tc_toep_launch(g, kTable, x, T, y, L));
+        if (st == WBMM_OK)
+            t_last_path = 1;
+        return st;
+    }
     if (dt == WBMM_BF16 && tc_fwd_supported(g, false)) {
         st = from_cuda(tc_fwd_launch(g, kTable, x, T, y, nullptr, L));
         if (st == WBMM_OK)
@@ -245,7 +251,10 @@ wbmm_status wbmm_backward(const void* x, const void* T, const void* dY, void* dX
     if ((st = make_launch(stream, &L)) != WBMM_OK)
         return st;
     if (dX) {
-        if (dt == WBMM_BF16 && tc_fwd_supported(g, false)) {
+        if (dt == WBMM_BF16 && tc_toep_supported(g)) {
+            st = from_cuda(tc_toep_launch(g, kTableFlip, dY, T, dX, L));
+            t_last_path = 1;
+        } else if (dt == WBMM_BF16 && tc_fwd_supported(g, false)) {
             st = from_cuda(tc_fwd_launch(g, kTableFlip, dY, T, dX, nullptr, L));
             t_last_path = 1;
         } else {

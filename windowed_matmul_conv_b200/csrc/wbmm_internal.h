@@ -58,6 +58,12 @@ bool tc_fwd_supported(const Geom& g, bool fused);
 cudaError_t tc_fwd_launch(const Geom& g, AMode mode, const void* x, const void* src, void* y,
                           const void* dw, const Launch& L);
 
+// tcgen05 forward / input gradient from the table, windows as the MMA's M
+// dimension (mode kTable or kTableFlip only).
+bool tc_toep_supported(const Geom& g);
+cudaError_t tc_toep_launch(const Geom& g, AMode mode, const void* x, const void* T, void* y,
+                           const Launch& L);
+
 // tcgen05 table gradient: per (channel, chunk) fp32 partial tables.
 bool tc_dt_supported(const Geom& g);
 int tc_dt_chunks(const Geom& g);
