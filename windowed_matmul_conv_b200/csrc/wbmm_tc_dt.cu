@@ -17,10 +17,13 @@
 // MN-major operand that layout has positions as M (or N) and windows as K,
 // so one thread issues 128 x NPOS x 16 MMAs (A = dY tile, B = x tile) into G
 // in TMEM (two 128-row halves when the padded positions exceed 128).  After
-// the item's last tile the epilogue warps read G from TMEM and add each entry
-// into a per-warp bin array in shared memory (within one TMEM column every
-// lane maps to a different bin, so the adds never collide), then sum the
-// four warp arrays in warp order into the item's partial table.
+// the item's last tile eight epilogue warps reduce G one 128-row half at a
+// time: every (p, r) block of G (image rows p and r, RP x RP entries) is
+// summed along its diagonals q - s in registers and written once to a
+// staging array [p][r][q - s]; the half is then released to the next item's
+// MMAs, and each thread adds the staged sums of the table entries it owns
+// (fixed p order) into registers.  The last half's sums are the item's
+// partial table.
 #include <cuda_bf16.h>
 
 #include "ptx_sm100.cuh"
@@ -32,18 +35,39 @@ namespace wbmm {
 constexpr uint32_t kSmemMax = 232448;
 constexpr int kDtRing = 2;
 constexpr int kDtXformWarps = 8;                 // warps 2..9
-constexpr int kDtEpiWarp0 = 2 + kDtXformWarps;  // warps 10..13
-constexpr int kDtThreads = (kDtEpiWarp0 + 4) * 32;
+constexpr int kDtEpiWarp0 = 2 + kDtXformWarps;  // warps 10..17
+constexpr int kDtEpiWarps = 8;
+constexpr int kDtEpiThreads = kDtEpiWarps * 32;
+constexpr int kDtThreads = (kDtEpiWarp0 + kDtEpiWarps) * 32;
+
+// Image rows p of G per 128-row half, and the staging array of one half:
+// fp32 [p][r][2*RP] with diagonal q - s = b at slot b + RP; the row of each p
+// is padded so that the 32/RP image rows a warp holds start RP banks apart
+// and one store instruction of the warp never conflicts.
+__host__ __device__ constexpr int dt_rows_per_half(int ws)
+{
+    const int pl = 128 / ((ws + 7) / 8 * 8);
+    return pl < ws ? pl : ws;
+}
+__host__ __device__ constexpr int dt_stg_stride(int ws)
+{
+    const int rp = (ws + 7) / 8 * 8;
+    return ws * 2 * rp + (rp - (ws * 2 * rp) % 32 + 32) % 32;
+}
+constexpr uint32_t dt_stg_bytes(int ws)
+{
+    return (uint32_t)(128 / ((ws + 7) / 8 * 8)) * dt_stg_stride(ws) * 4;
+}
 
 // Shared memory of the dT kernel for window size ws and nt windows per tile:
-// two operand stages (dY and x tiles), the raw ring, per-warp bins, barriers.
+// two operand stages (dY and x tiles), the raw ring, the staging array,
+// barriers.
 constexpr uint32_t dt_smem_bytes(int ws, int nt)
 {
     const int d = ws * ws, rp = (ws + 7) / 8 * 8, kp = (ws * rp + 15) / 16 * 16;
     const uint32_t stage = 2u * (uint32_t)nt * kp * 2;
     const uint32_t raw = 2u * (uint32_t)((nt * d * 2 + 127) / 128 * 128);
-    const uint32_t bins = 4u * (2 * ws - 1) * (2 * ws - 1) * 4;
-    return 2 * stage + kDtRing * raw + bins + nt * 4 + 2048;
+    return 2 * stage + kDtRing * raw + dt_stg_bytes(ws) + nt * 4 + 2048;
 }
 
 // Windows per tile: 64 when the layout fits, else 32 (w >= 15).
@@ -80,7 +104,7 @@ struct TcDtParams {
     int items;              // C * chunks
     int use_tmap;           // tiles are whole planes: one 4-D TMA per tensor
     int kimg;               // planes per tile when use_tmap
-    uint32_t off_raw, off_stage, off_bins, off_woff, off_bar;
+    uint32_t off_raw, off_stage, off_stg, off_woff, off_bar;
     unsigned long long budget;
     int* status;
 };
@@ -91,7 +115,7 @@ struct DtBars {
     uint64_t st_full[2];
     uint64_t st_empty[2];
     uint64_t g_full;
-    uint64_t g_empty;
+    uint64_t g_empty[2];    // per 128-row half of G
     uint64_t fin;
     uint32_t tmem_slot;
     int abort;
@@ -150,7 +174,7 @@ __global__ void __launch_bounds__(kDtThreads, 1) wbmm_tc_dt_kernel(const __grid_
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     uint8_t* raw_base = smem + P.off_raw;
     uint8_t* st_base = smem + P.off_stage;
-    float* bins = reinterpret_cast<float*>(smem + P.off_bins);
+    float* stg = reinterpret_cast<float*>(smem + P.off_stg);
     int* woff = reinterpret_cast<int*>(smem + P.off_woff);
     DtBars& S = *reinterpret_cast<DtBars*>(smem + P.off_bar);
     volatile int* abort = &S.abort;
@@ -165,7 +189,8 @@ __global__ void __launch_bounds__(kDtThreads, 1) wbmm_tc_dt_kernel(const __grid_
             mbar_init(&S.st_empty[i], 1);
         }
         mbar_init(&S.g_full, 1);
-        mbar_init(&S.g_empty, 4);
+        mbar_init(&S.g_empty[0], kDtEpiWarps);
+        mbar_init(&S.g_empty[1], kDtEpiWarps);
         mbar_init(&S.fin, 1);
         S.abort = 0;
         fence_mbar_init();
@@ -245,22 +270,25 @@ __global__ void __launch_bounds__(kDtThreads, 1) wbmm_tc_dt_kernel(const __grid_
                 const DtTile t = it.get(P);
                 const int bs = seq & 1;
                 bool ok = !*abort;
-                if (t.first) {
+                if (t.first)
                     ok_item = true;
-                    if (item_seq > 0)
-                        ok = ok && mbar_wait(&S.g_empty, (item_seq - 1) & 1, abort, P.budget,
-                                             P.status);
-                }
                 ok = ok && mbar_wait(&S.st_full[bs], (seq >> 1) & 1, abort, P.budget, P.status);
                 ok_item = ok_item && ok;
                 if (ok) {
-                    tc_fence_after();
                     const uint32_t a_addr = smem_u32(st_base + (size_t)bs * F::STAGE_BYTES);
                     const uint32_t b_addr = a_addr + F::TILE_BYTES;
                     const int nwin = t.bt.nb * P.nw;
                     const int ksteps = (nwin + 15) >> 4;
 #pragma unroll
                     for (int mt = 0; mt < F::MT; ++mt) {
+                        // the previous item's reduction hands G over one
+                        // 128-row half at a time
+                        if (t.first && item_seq > 0)
+                            ok = ok && mbar_wait(&S.g_empty[mt], (item_seq - 1) & 1, abort,
+                                                 P.budget, P.status);
+                        if (!ok)
+                            break;
+                        tc_fence_after();
 #pragma unroll 1
                         for (int k = 0; k < ksteps; ++k) {
                             // MN-major: LBO = window-group stride, SBO = position-group stride
@@ -272,7 +300,9 @@ __global__ void __launch_bounds__(kDtThreads, 1) wbmm_tc_dt_kernel(const __grid_
                                    (t.first && k == 0) ? 0u : 1u);
                         }
                     }
-                    tc_commit(&S.st_empty[bs]);
+                    if (ok)
+                        tc_commit(&S.st_empty[bs]);
+                    ok_item = ok_item && ok;
                 }
                 if (t.last) {
                     if (ok_item)
@@ -317,114 +347,116 @@ __global__ void __launch_bounds__(kDtThreads, 1) wbmm_tc_dt_kernel(const __grid_
         }
     } else {
         // ------------------------------------------------------ epilogue
+        // Two warps per TMEM lane quarter; warp half h takes the 32-column
+        // chunks h, h+2, ... of its 32 rows of G.  With positions padded to
+        // RP slots per image row, the 32 lanes are 32/RP segments of one image
+        // row p each, and a chunk is 32/RP blocks of one column row r each.
+        // The diagonal sums of an RP x RP block (fixed p, r) come from
+        // width-RP shuffles: lane L takes column s from lane (L+s)%RP, an
+        // entry of diagonal q - s = L (no wrap) or L - RP (wrap), and adds it
+        // to one of two sums in ascending s; both sums are staged with
+        // unconditional stores (slots of invalid diagonals are never read).
+        // Columns s >= w are zero padding and are skipped.
+        constexpr int RP = F::RP;
+        constexpr int NB = 32 / RP;                  // blocks (r values) per chunk
+        constexpr int NCH = (F::NPOS + 31) / 32;     // chunks per row (last may overhang)
+        constexpr int L2 = 2 * WS - 1;
+        constexpr int PL = dt_rows_per_half(WS);     // image rows p per half
+        constexpr int SP = dt_stg_stride(WS);        // staging floats per image row p
+        constexpr int NBT = (F::TSZ + kDtEpiThreads - 1) / kDtEpiThreads;
         const int quarter = warp & 3;
-        const int ew = warp - kDtEpiWarp0;
+        const int h = (warp - kDtEpiWarp0) >> 2;
         const int et = threadIdx.x - kDtEpiWarp0 * 32;
-        float* mybins = bins + ew * F::TSZ;
+        const int L = lane & (RP - 1);
         int item_seq = 0;
         for (int item = blockIdx.x; item < P.items; item += gridDim.x, ++item_seq) {
             bool ok = !*abort;
             ok = ok && mbar_wait(&S.g_full, item_seq & 1, abort, P.budget, P.status);
             ok = __all_sync(0xffffffffu, ok);
             tc_fence_after();
-            for (int i = lane; i < F::TSZ; i += 32)
-                mybins[i] = 0.0f;
-            __syncwarp();
-            if (ok) {
-                // This warp reads rows u = mt*128 + quarter*32 + lane of G; with
-                // positions padded to RP slots per window row, the 32 lanes are
-                // 32/RP segments of one image row p each, and a 32-column TMEM
-                // chunk is 32/RP blocks of one column row r each.  The
-                // diagonal sums of a RP x RP block (fixed p, r) come from RP
-                // width-RP shuffles: lane L takes column s from lane (L+s)%RP,
-                // an entry of diagonal dq = L (no wrap) or dq = L - RP (wrap);
-                // fixed-shape tree sums give each lane the two diagonal sums of
-                // every block, kept in registers until the pass ends and then
-                // added to the bins of rows dp = p - r, one segment at a time.
-                constexpr int RP = F::RP;
-                constexpr int NB = 32 / RP;             // blocks (r values) per chunk
-                constexpr int NCH = (F::NPOS + 31) / 32;    // chunks per row (last may overhang)
-                const int L = lane & (RP - 1);
+            float acc[NBT];
+#pragma unroll
+            for (int i = 0; i < NBT; ++i)
+                acc[i] = 0.0f;
 #pragma unroll 1
-                for (int mt = 0; mt < F::MT; ++mt) {
-                    const int ubase = mt * 128 + quarter * 32;
-                    const int p = (ubase + lane) / RP;
-                    if (ubase / RP >= WS)
-                        break;                           // warp-uniform: only padding rows left
+            for (int mt = 0; mt < F::MT; ++mt) {
+                const int ubase = mt * 128 + quarter * 32;
+                // warp-uniform: rows past the last image row are padding
+                if (ok && ubase / RP < WS && h < NCH) {
                     const uint32_t gcol =
                         tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(mt * 256);
-                    float dsum[WS][2];
-#pragma unroll
-                    for (int rr = 0; rr < WS; ++rr)
-                        dsum[rr][0] = dsum[rr][1] = 0.0f;
-                    uint32_t r[32];
-                    tmem_ld32(gcol, r);
-#pragma unroll
-                    for (int ch = 0; ch < NCH; ++ch) {
+#pragma unroll 1
+                    for (int ch = h; ch < NCH; ch += 2) {
+                        uint32_t r[32];
+                        tmem_ld32(gcol + (uint32_t)(ch * 32), r);
                         tmem_wait_ld(r);
                         float v[32];
 #pragma unroll
                         for (int jj = 0; jj < 32; ++jj)
                             v[jj] = __uint_as_float(r[jj]);
-                        if (ch + 1 < NCH)
-                            tmem_ld32(gcol + (uint32_t)((ch + 1) * 32), r);   // next chunk in flight
 #pragma unroll
                         for (int b = 0; b < NB; ++b) {
                             const int rr = ch * NB + b;
                             if (rr < WS) {
-                                float a[RP], c[RP];
+                                float a = 0.0f, c = 0.0f;
 #pragma unroll
-                                for (int s = 0; s < RP; ++s) {
+                                for (int s = 0; s < WS; ++s) {
                                     const float g = __shfl_sync(0xffffffffu, v[b * RP + s],
                                                                 (L + s) & (RP - 1), RP);
-                                    const bool in_a = L + s < RP;
-                                    a[s] = in_a ? g : 0.0f;
-                                    c[s] = in_a ? 0.0f : g;
+                                    if (L + s < RP)
+                                        a += g;
+                                    else
+                                        c += g;
                                 }
-#pragma unroll
-                                for (int h = RP / 2; h >= 1; h /= 2)
-#pragma unroll
-                                    for (int s = 0; s < h; ++s) {
-                                        a[s] = a[s] + a[s + h];
-                                        c[s] = c[s] + c[s + h];
-                                    }
-                                dsum[rr][0] = a[0];
-                                dsum[rr][1] = c[0];
+                                float* row = stg + ((ubase - mt * 128 + lane) / RP) * SP + rr * 2 * RP;
+                                row[L + RP] = a;
+                                row[L] = c;
                             }
                         }
-                    }
-#pragma unroll
-                    for (int seg = 0; seg < 32 / RP; ++seg) {
-                        if (lane / RP == seg && p < WS) {
-#pragma unroll
-                            for (int rr = 0; rr < WS; ++rr) {
-                                const int row = (p - rr + WS - 1) * (2 * WS - 1) + (WS - 1);
-                                if (L <= WS - 1)
-                                    mybins[row + L] += dsum[rr][0];
-                                if (L - RP >= -(WS - 1))
-                                    mybins[row + L - RP] += dsum[rr][1];
-                            }
-                        }
-                        __syncwarp();
                     }
                 }
+                // this half of G has been read: the next item's MMAs may
+                // overwrite it while the staged sums are added up
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(&S.g_empty[mt]);
+                named_bar_sync(3, kDtEpiThreads);
+                if (ok) {
+                    // the thread's bins are independent chains: interleave them
+                    int da[NBT], off[NBT];
+#pragma unroll
+                    for (int i = 0; i < NBT; ++i) {
+                        const int bin = et + i * kDtEpiThreads;
+                        const int bb = bin < F::TSZ ? bin : 0;
+                        da[i] = bin < F::TSZ ? bb / L2 - (WS - 1) : 4 * WS;   // out of range: no adds
+                        off[i] = bb - (bb / L2) * L2 - (WS - 1) + RP;
+                    }
+                    const int p0 = mt * PL;
+#pragma unroll
+                    for (int j = 0; j < PL; ++j) {
+                        const int pp = p0 + j;
+                        if (pp < WS) {
+#pragma unroll
+                            for (int i = 0; i < NBT; ++i) {
+                                const int rr = pp - da[i];
+                                if (rr >= 0 && rr < WS)
+                                    acc[i] += stg[j * SP + rr * 2 * RP + off[i]];
+                            }
+                        }
+                    }
+                }
+                named_bar_sync(3, kDtEpiThreads);
             }
-            tc_fence_before();
-            __syncwarp();
-            if (ok && lane == 0)
-                mbar_arrive(&S.g_empty);
-            named_bar_sync(3, 128);
             if (ok) {
                 float* out = P.partials + (long long)item * F::TSZ;
-                for (int i = et; i < F::TSZ; i += 128) {
-                    float acc = bins[i];
-                    acc += bins[F::TSZ + i];
-                    acc += bins[2 * F::TSZ + i];
-                    acc += bins[3 * F::TSZ + i];
-                    out[i] = acc;
+#pragma unroll
+                for (int i = 0; i < NBT; ++i) {
+                    const int bin = et + i * kDtEpiThreads;
+                    if (bin < F::TSZ)
+                        out[bin] = acc[i];
                 }
             }
-            named_bar_sync(3, 128);
         }
     }
 
@@ -444,7 +476,7 @@ constexpr uint32_t kMinSmem = 120 * 1024;
 inline uint32_t align_up(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
 
 struct DtLayout {
-    uint32_t off_raw, off_stage, off_bins, off_woff, off_bar, total;
+    uint32_t off_raw, off_stage, off_stg, off_woff, off_bar, total;
 };
 
 template <int WS>
@@ -457,8 +489,8 @@ DtLayout dt_layout()
     off += 2 * F::STAGE_BYTES;
     L.off_raw = align_up(off, 128);
     off = L.off_raw + kDtRing * F::RAW_BYTES;
-    L.off_bins = align_up(off, 16);
-    off = L.off_bins + 4 * F::TSZ * 4;
+    L.off_stg = align_up(off, 16);
+    off = L.off_stg + dt_stg_bytes(WS);
     L.off_woff = align_up(off, 16);
     off = L.off_woff + F::NT * 4;
     L.off_bar = align_up(off, 16);
@@ -518,7 +550,7 @@ cudaError_t dt_launch_ws(const Geom& g, const void* x, const void* dy, float* pa
             P.kimg = k;
         }
     }
-    P.off_raw = lay.off_raw; P.off_stage = lay.off_stage; P.off_bins = lay.off_bins;
+    P.off_raw = lay.off_raw; P.off_stage = lay.off_stage; P.off_stg = lay.off_stg;
     P.off_woff = lay.off_woff; P.off_bar = lay.off_bar;
     P.budget = L.budget;
     P.status = L.status;
