@@ -190,12 +190,20 @@ class Arm:
                 s["z"] = torch.empty_like(s["x"])
 
     def kernels(self):
+        """The step's kernels, one call each (the per-kernel breakdown)."""
         k = self.wl.kind
         if k == "train":
             return ["forward", "backward_dx", "backward_dt"]
         if k == "cached_dw":
             return ["forward_cached", "dw3x3"]
         return ["forward"]
+
+    def calls(self):
+        """The step as a user issues it: the training step is one forward
+        and one backward call that returns both dX and dT."""
+        if self.wl.kind == "train":
+            return ["forward", "backward"]
+        return self.kernels()
 
     def launch(self, name, s):
         wb, w = self.wb, self.wl.w
@@ -205,6 +213,8 @@ class Arm:
             wb.wbmm_backward(None, self.T, s["dY"], s["dX"], None, None, w)
         elif name == "backward_dt":
             wb.wbmm_backward(s["x"], None, s["dY"], None, self.dT, self.ws, w)
+        elif name == "backward":
+            wb.wbmm_backward(s["x"], self.T, s["dY"], s["dX"], self.dT, self.ws, w)
         elif name == "forward_cached":
             wb.wbmm_forward_cached(s["x"], self.M, None, s["y"], w)
         elif name == "dw3x3":
@@ -212,7 +222,7 @@ class Arm:
 
     def step(self, k):
         s = self.sets[k % len(self.sets)]
-        for name in self.kernels():
+        for name in self.calls():
             self.launch(name, s)
 
 
@@ -335,7 +345,7 @@ def run_gpu(args, rank, world, local_rank):
     ms_total = max_over_ranks(e0.elapsed_time(e1), world, dev)
     ms_step = ms_total / K
     # graph replays launch the captured kernels: count them per step
-    per_step_launches = len(wb_arm.kernels()) + (1 if wl.kind == "train" else 0)
+    per_step_launches = len(wb_arm.kernels())
     gpu_launches = per_step_launches * K
     assert wb.wbmm_launch_count() == launches0   # graphs: no host launches
 

@@ -63,13 +63,20 @@ def test_workspace_size_formula(lib):
     f = lib.wbmm_backward_workspace_bytes
     f.restype = ctypes.c_size_t
     f.argtypes = [ctypes.c_int] * 6
+    # bf16, tensor-core path: one partial table per (channel, CTA range)
+    # segment, at most n = C + min(256, tiles) - 1 of them, then one 64-bit
+    # flag per table (8-byte aligned).
+    def tc(n, tsz=729):
+        return ((n * tsz + 1) // 2 * 2 + 2 * n) * 4
     # training workload: 64-window tiles of 32 two-window bands, 8 tiles per
-    # channel, one chunk of up to 16 tiles -> 1 fp32 partial table per channel
-    assert f(128, 256, 28, 28, 14, 1) == 256 * 1 * 729 * 4
-    # 64 images of 56x56: 16 bands/tile, 16 tiles/channel -> 1 chunk
-    assert f(64, 128, 56, 56, 14, 1) == 128 * 1 * 729 * 4
-    # 32 images of 112x112: 8 bands/tile, 32 tiles/channel -> 2 chunks
-    assert f(32, 4, 112, 112, 14, 1) == 4 * 2 * 729 * 4
+    # channel, 2048 tiles -> 256 + 255 tables
+    assert f(128, 256, 28, 28, 14, 1) == tc(256 + 255)
+    # 64 images of 56x56: 16 bands/tile, 16 tiles/channel, 2048 tiles
+    assert f(64, 128, 56, 56, 14, 1) == tc(128 + 255)
+    # 32 images of 112x112: 8 bands/tile, 32 tiles/channel, 128 tiles
+    assert f(32, 4, 112, 112, 14, 1) == tc(4 + 127)
+    # fp32, CUDA-core path: chunks of 8 bands per channel
+    assert f(2, 3, 14, 28, 7, 0) == 3 * 1 * 169 * 4
     assert f(1, 1, 14, 15, 7, 1) == 0
 
 

@@ -121,6 +121,41 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t *bar, uint32_t parity,
     return true;
 }
 
+// ------------------------------------------------ flags between CTAs
+__device__ __forceinline__ void st_release_u64(unsigned long long *p, unsigned long long v)
+{
+    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long *p)
+{
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Bounded wait until *p == token (written by another CTA of the same grid).
+// Gives up on the abort flag or after `budget` SM cycles; in the second case
+// it raises the abort flag and the device status word.  Returns true when the
+// token arrived.
+__device__ __forceinline__ bool wait_token(const unsigned long long *p, unsigned long long token,
+                                           volatile int *abort, unsigned long long budget,
+                                           int *status)
+{
+    const long long t0 = clock64();
+    while (ld_acquire_u64(p) != token) {
+        if (*abort)
+            return false;
+        if ((unsigned long long)(clock64() - t0) > budget) {
+            *abort = 1;
+            atomicOr(status, kStatusTimeout);
+            return false;
+        }
+        __nanosleep(256);
+    }
+    return true;
+}
+
 // ------------------------------------------------------- bulk async copies
 // Global -> shared, completion signalled on `bar` as transaction bytes.
 // Both addresses 16-byte aligned, bytes a multiple of 16.

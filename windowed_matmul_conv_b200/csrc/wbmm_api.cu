@@ -119,12 +119,12 @@ size_t map_bytes(const Geom& g, wbmm_dtype dt)
     return (size_t)g.B * g.C * g.H * g.W * elem_size(dt);
 }
 
-// Partial-table chunks the backward will use for this shape and dtype.
-int dt_chunks_for(const Geom& g, wbmm_dtype dt)
+// Workspace floats the backward will use for this shape and dtype.
+long long dt_workspace_floats(const Geom& g, wbmm_dtype dt)
 {
     if (dt == WBMM_BF16 && tc_dt_supported(g))
-        return tc_dt_chunks(g);
-    return simt_dt_chunks(g);
+        return tc_dt_workspace_floats(g);
+    return (long long)g.C * simt_dt_chunks(g) * g.tsz;
 }
 
 }  // namespace
@@ -207,7 +207,7 @@ size_t wbmm_backward_workspace_bytes(int B, int C, int H, int W, int w, wbmm_dty
     if (!dtype_ok(dt) || check_map(B, C, H, W, w) != WBMM_OK)
         return 0;
     const Geom g = make_geom(B, C, H, W, w);
-    return (size_t)C * dt_chunks_for(g, dt) * g.tsz * sizeof(float);
+    return (size_t)dt_workspace_floats(g, dt) * sizeof(float);
 }
 
 wbmm_status wbmm_backward(const void* x, const void* T, const void* dY, void* dX, float* dT,
@@ -250,6 +250,7 @@ wbmm_status wbmm_backward(const void* x, const void* T, const void* dY, void* dX
     Launch L;
     if ((st = make_launch(stream, &L)) != WBMM_OK)
         return st;
+    const bool tc_dt = dT && dt == WBMM_BF16 && tc_dt_supported(g);
     if (dX) {
         if (dt == WBMM_BF16 && tc_toep_supported(g)) {
             st = from_cuda(tc_toep_launch(g, kTableFlip, dY, T, dX, L));
@@ -266,14 +267,17 @@ wbmm_status wbmm_backward(const void* x, const void* T, const void* dY, void* dX
     }
     if (dT) {
         float* part = static_cast<float*>(workspace);
-        const int chunks = dt_chunks_for(g, dt);
-        if (dt == WBMM_BF16 && tc_dt_supported(g))
-            st = from_cuda(tc_dt_launch(g, x, dY, part, L));
-        else
+        if (tc_dt) {
+            // dX, when requested, was the launch just before this one (every
+            // library kernel signals its dependents only after its own wait)
+            const bool after_dx = dX != nullptr;
+            st = from_cuda(tc_dt_launch(g, x, dY, part, dT, after_dx, L));
+        } else {
             st = from_cuda(simt_dt_launch(g, dt == WBMM_BF16, x, dY, part, L));
-        if (st != WBMM_OK)
-            return st;
-        st = from_cuda(dt_finalize_launch(C, g.tsz, chunks, part, dT, L));
+            if (st != WBMM_OK)
+                return st;
+            st = from_cuda(dt_finalize_launch(C, g.tsz, simt_dt_chunks(g), part, dT, L));
+        }
     }
     return st;
 }

@@ -64,11 +64,17 @@ bool tc_toep_supported(const Geom& g);
 cudaError_t tc_toep_launch(const Geom& g, AMode mode, const void* x, const void* T, void* y,
                            const Launch& L);
 
-// tcgen05 table gradient: per (channel, chunk) fp32 partial tables.
+// tcgen05 table gradient: one contiguous tile range per CTA.  The workspace
+// (tc_dt_workspace_floats floats, any prior content) holds the fp32 partial
+// tables of channels split between CTAs and one flag word per table.
+// after_dx: the previous launch on the stream is the same backward call's
+// input-gradient kernel (which reads dY and T and writes only dX), so the
+// kernel need not wait for it to finish.
 bool tc_dt_supported(const Geom& g);
-int tc_dt_chunks(const Geom& g);
-cudaError_t tc_dt_launch(const Geom& g, const void* x, const void* dy, float* partials,
-                         const Launch& L);
+long long tc_dt_partials(const Geom& g);
+long long tc_dt_workspace_floats(const Geom& g);
+cudaError_t tc_dt_launch(const Geom& g, const void* x, const void* dy, float* workspace, float* dT,
+                         bool after_dx, const Launch& L);
 
 // CUDA-core kernels.  is_bf16 selects the element type of every map/table.
 int simt_dt_chunks(const Geom& g);

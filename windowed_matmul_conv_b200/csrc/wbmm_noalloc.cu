@@ -84,8 +84,8 @@ extern "C" WBMM_API wbmm_status wbmm_backward_dt_static(const void* x, const voi
     }
     // Same partial-table split as wbmm_backward, checked against the array.
     const bool tc = dt == WBMM_BF16 && tc_dt_supported(g);
-    const int chunks = tc ? tc_dt_chunks(g) : simt_dt_chunks(g);
-    if ((size_t)C * chunks * g.tsz > kStaticPartials)
+    const long long need = tc ? tc_dt_workspace_floats(g) : (long long)C * simt_dt_chunks(g) * g.tsz;
+    if ((unsigned long long)need > kStaticPartials)
         return WBMM_ERR_WORKSPACE;
 
     float* part = nullptr;
@@ -96,10 +96,14 @@ extern "C" WBMM_API wbmm_status wbmm_backward_dt_static(const void* x, const voi
     if ((st = static_cast<wbmm_status>(launch_for_stream(stream, &L))) != WBMM_OK)
         return st;
 
-    cudaError_t e = tc ? tc_dt_launch(g, x, dY, part, L)
-                       : simt_dt_launch(g, dt == WBMM_BF16, x, dY, part, L);
-    if (e == cudaSuccess)
-        e = dt_finalize_launch(C, g.tsz, chunks, part, dT, L);
+    cudaError_t e;
+    if (tc) {
+        e = tc_dt_launch(g, x, dY, part, dT, false, L);
+    } else {
+        e = simt_dt_launch(g, dt == WBMM_BF16, x, dY, part, L);
+        if (e == cudaSuccess)
+            e = dt_finalize_launch(C, g.tsz, simt_dt_chunks(g), part, dT, L);
+    }
     if (e == cudaErrorInvalidConfiguration)
         return WBMM_ERR_UNSUPPORTED;
     return e == cudaSuccess ? WBMM_OK : WBMM_ERR_CUDA;

@@ -6,10 +6,19 @@
 // and the table gradient is its sum along constant relative offset:
 //   dT[(p-r+w-1)(2w-1) + (q-s+w-1)] = sum over (u=(p,q), v=(r,s)) of G[u, v].
 //
-// Work item = (channel, fixed chunk of tiles).  The chunk split depends only
-// on the shape, every sum runs in a fixed order, and each item writes its own
-// fp32 partial table, so the result is bit-identical from run to run and for
-// any grid size; a second kernel adds the partials in chunk order.
+// The channels' tiles, in channel order, are split into one contiguous,
+// balanced range per CTA.  A segment is the part of a CTA's range inside one
+// channel; each segment ends with one reduction of G into its own fp32 partial
+// table, at index c + k (channel c, CTA k: ranges are ordered, so the index
+// is unique).  A channel inside one CTA's range is written to dT directly.
+// A channel split between CTAs k0 < ... < k1 is the last segment of CTA k0
+// and an earlier segment of every later one: those write their partial table
+// and then a flag word holding this launch's 64-bit token (release); k0 waits
+// for the flags (bounded) and adds its own sums and then the later partials,
+// in CTA order, into dT.  Stale flags hold other launches' tokens, so the
+// workspace needs no initialisation.  Every sum runs in a fixed order, so the
+// result is bit-identical from run to run for a given grid (the device's SM
+// count).
 //
 // Per tile the producer bulk-copies the dY and x bands into a raw slot; the
 // transform warps write both tiles in the layout of the forward kernel's
@@ -17,14 +26,17 @@
 // MN-major operand that layout has positions as M (or N) and windows as K,
 // so one thread issues 128 x NPOS x 16 MMAs (A = dY tile, B = x tile) into G
 // in TMEM (two 128-row halves when the padded positions exceed 128).  After
-// the item's last tile eight epilogue warps reduce G one 128-row half at a
+// the segment's last tile eight epilogue warps reduce G one 128-row half at a
 // time: every (p, r) block of G (image rows p and r, RP x RP entries) is
 // summed along its diagonals q - s in registers and written once to a
-// staging array [p][r][q - s]; the half is then released to the next item's
+// staging array [p][r][q - s]; the half is then released to the next segment's
 // MMAs, and each thread adds the staged sums of the table entries it owns
-// (fixed p order) into registers.  The last half's sums are the item's
+// (fixed p order) into registers.  The last half's sums are the segment's
 // partial table.
 #include <cuda_bf16.h>
+
+#include <atomic>
+#include <chrono>
 
 #include "ptx_sm100.cuh"
 #include "tc_common.cuh"
@@ -94,14 +106,17 @@ struct TcDtParams {
     TmapBytes map_dy;
     const uint16_t* x;
     const uint16_t* dy;
-    float* partials;        // [C][chunks][tsz]
+    float* partials;        // [C + grid - 1][tsz], segment (c, k) at c + k
+    unsigned long long* flags;  // [C + grid - 1], token when partial c + k is written
+    unsigned long long token;   // unique per launch
+    float* dT;              // [C][tsz]
     int C, H, W, nh, nw;
     int bpt;
     int tpc;                // tiles per channel
-    int ch;                 // tiles per chunk
-    int chunks;             // chunks per channel
     int bands;
-    int items;              // C * chunks
+    int rq, rr;             // range split: CTA k gets rq + (k < rr) tiles
+    int dep_wait;           // 0: the previous kernel reads only what this one
+                            // reads and writes nothing it touches
     int use_tmap;           // tiles are whole planes: one 4-D TMA per tensor
     int kimg;               // planes per tile when use_tmap
     uint32_t off_raw, off_stage, off_stg, off_woff, off_bar;
@@ -119,51 +134,51 @@ struct DtBars {
     uint64_t fin;
     uint32_t tmem_slot;
     int abort;
+    int seg_ok;             // the later segments of the current channel arrived
 };
 
 struct DtTile {
     BandTile bt;
-    bool first, last;   // first / last tile of its item
+    bool first, last;   // first / last tile of its segment
 };
 
-// The flattened tile sequence of a CTA: items blockIdx.x, +grid, ...; within
-// an item its tiles in order.  Every role walks the same sequence.
+// The CTA whose range holds tile t (inverse of dt_range).
+__device__ __forceinline__ int dt_cta_of(const TcDtParams& P, long long t)
+{
+    const long long big = (long long)P.rr * (P.rq + 1);
+    return (int)(t < big ? t / (P.rq + 1) : P.rr + (t - big) / P.rq);
+}
+
+// The tile range of a CTA: [t0, t1) of the channel-major tile sequence.
+__device__ __forceinline__ void dt_range(const TcDtParams& P, int& t0, int& t1)
+{
+    const int k = (int)blockIdx.x;
+    t0 = k * P.rq + (k < P.rr ? k : P.rr);
+    t1 = t0 + P.rq + (k < P.rr ? 1 : 0);
+}
+
+// Every role walks the CTA's range in the same order.
 struct DtWalker {
-    int item;
-    int tile;       // tile index within the channel
-    int tile0, tile_end;
-    __device__ __forceinline__ bool valid(const TcDtParams& P) const { return item < P.items; }
+    int t, t0, t1;
+    __device__ __forceinline__ bool valid(const TcDtParams&) const { return t < t1; }
     __device__ __forceinline__ void start(const TcDtParams& P)
     {
-        item = blockIdx.x;
-        set_item(P);
-    }
-    __device__ __forceinline__ void set_item(const TcDtParams& P)
-    {
-        if (item >= P.items)
-            return;
-        tile0 = (item % P.chunks) * P.ch;
-        tile = tile0;
-        tile_end = tile0 + P.ch < P.tpc ? tile0 + P.ch : P.tpc;
+        dt_range(P, t0, t1);
+        t = t0;
     }
     __device__ __forceinline__ DtTile get(const TcDtParams& P) const
     {
-        DtTile t;
-        t.bt.c = item / P.chunks;
-        t.bt.band0 = tile * P.bpt;
-        const int left = P.bands - t.bt.band0;
-        t.bt.nb = left < P.bpt ? left : P.bpt;
-        t.first = tile == tile0;
-        t.last = tile + 1 == tile_end;
-        return t;
+        DtTile d;
+        d.bt.c = t / P.tpc;
+        const int tile = t - d.bt.c * P.tpc;
+        d.bt.band0 = tile * P.bpt;
+        const int left = P.bands - d.bt.band0;
+        d.bt.nb = left < P.bpt ? left : P.bpt;
+        d.first = t == t0 || tile == 0;
+        d.last = t + 1 == t1 || tile + 1 == P.tpc;
+        return d;
     }
-    __device__ __forceinline__ void next(const TcDtParams& P)
-    {
-        if (++tile >= tile_end) {
-            item += gridDim.x;
-            set_item(P);
-        }
-    }
+    __device__ __forceinline__ void next(const TcDtParams&) { ++t; }
 };
 
 template <int WS>
@@ -212,8 +227,12 @@ __global__ void __launch_bounds__(kDtThreads, 1) wbmm_tc_dt_kernel(const __grid_
     tc_fence_after();
     const uint32_t tmem = S.tmem_slot;
     // Everything above overlaps the previous kernel's tail; tensors are read
-    // and written only after it has completed.
-    grid_dep_wait();
+    // and written only after it has completed.  The input-gradient kernel of
+    // the same backward call is the exception: it signals this launch only
+    // after its own wait, so whatever produced dY and x is complete, and it
+    // writes nothing this kernel touches.
+    if (P.dep_wait)
+        grid_dep_wait();
     grid_dep_launch();
 
     if (warp == 0) {
@@ -368,8 +387,11 @@ __global__ void __launch_bounds__(kDtThreads, 1) wbmm_tc_dt_kernel(const __grid_
         const int h = (warp - kDtEpiWarp0) >> 2;
         const int et = threadIdx.x - kDtEpiWarp0 * 32;
         const int L = lane & (RP - 1);
+        int t0, t1;
+        dt_range(P, t0, t1);
+        const int c_first = t0 / P.tpc, c_last = (t1 - 1) / P.tpc;
         int item_seq = 0;
-        for (int item = blockIdx.x; item < P.items; item += gridDim.x, ++item_seq) {
+        for (int c = c_first; c <= c_last; ++c, ++item_seq) {
             bool ok = !*abort;
             ok = ok && mbar_wait(&S.g_full, item_seq & 1, abort, P.budget, P.status);
             ok = __all_sync(0xffffffffu, ok);
@@ -448,15 +470,61 @@ __global__ void __launch_bounds__(kDtThreads, 1) wbmm_tc_dt_kernel(const __grid_
                 }
                 named_bar_sync(3, kDtEpiThreads);
             }
-            if (ok) {
-                float* out = P.partials + (long long)item * F::TSZ;
+            const int k0 = dt_cta_of(P, (long long)c * P.tpc);
+            const int k1 = dt_cta_of(P, (long long)c * P.tpc + P.tpc - 1);
+            if (k0 == k1) {
+                // the whole channel is in this CTA's range
+                if (ok) {
+                    float* out = P.dT + (long long)c * F::TSZ;
+#pragma unroll
+                    for (int i = 0; i < NBT; ++i) {
+                        const int bin = et + i * kDtEpiThreads;
+                        if (bin < F::TSZ)
+                            out[bin] = acc[i];
+                    }
+                }
+                continue;
+            }
+            const int k = (int)blockIdx.x;
+            if (k != k0) {
+                // an earlier segment of this CTA: publish it for CTA k0
+                float* out = P.partials + (long long)(c + k) * F::TSZ;
 #pragma unroll
                 for (int i = 0; i < NBT; ++i) {
                     const int bin = et + i * kDtEpiThreads;
                     if (bin < F::TSZ)
                         out[bin] = acc[i];
                 }
+                __threadfence();
+                named_bar_sync(3, kDtEpiThreads);
+                if (et == 0)
+                    st_release_u64(P.flags + c + k, P.token);
+                continue;
             }
+            // this CTA holds the channel's first tiles and its last segment:
+            // wait for the later segments, then add them in CTA order
+            if (et == 0) {
+                int good = 1;
+                for (int kk = k0 + 1; kk <= k1 && good; ++kk)
+                    good = wait_token(P.flags + c + kk, P.token, abort, P.budget, P.status);
+                S.seg_ok = good;
+            }
+            named_bar_sync(3, kDtEpiThreads);
+            if (ok && S.seg_ok) {
+                __threadfence();
+#pragma unroll
+                for (int i = 0; i < NBT; ++i) {
+                    const int bin = et + i * kDtEpiThreads;
+                    if (bin < F::TSZ) {
+                        const float* pc = P.partials + (long long)c * F::TSZ + bin;
+                        float sum = acc[i];
+                        for (int kk = k0 + 1; kk <= k1; ++kk)
+                            sum += __ldcg(pc + (long long)kk * F::TSZ);
+                        P.dT[(long long)c * F::TSZ + bin] = sum;
+                    }
+                }
+            }
+            named_bar_sync(3, kDtEpiThreads);   // seg_ok is rewritten next
         }
     }
 
@@ -503,17 +571,50 @@ DtLayout dt_layout()
     return L;
 }
 
-// Tiles per chunk: a fixed function of the shape (never of the grid).  Each
-// chunk ends with one reduction of G, so chunks are as long as the channel
-// allows, up to 16 tiles.
-int chunk_tiles(int tpc)
+// Largest grid of the table-gradient kernel: bounds the number of partial
+// tables (C + grid - 1) without knowing the device.
+constexpr int kDtMaxGrid = 256;
+
+long long tc_dt_partials_impl(const Geom& g);
+
+// Float offset of the flag words in the workspace (after the partial tables,
+// rounded up to 8 bytes).
+long long dt_flags_offset(const Geom& g)
 {
-    return tpc < 16 ? tpc : 16;
+    return (tc_dt_partials_impl(g) * g.tsz + 1) / 2 * 2;
+}
+
+// A token no earlier launch of this process used; the start is drawn from
+// the clock and the address space so that another process's stale flags
+// match with probability ~2^-64.
+unsigned long long next_launch_token()
+{
+    static std::atomic<unsigned long long> ctr{0};
+    static const unsigned long long seed = [] {
+        unsigned long long v = (unsigned long long)std::chrono::steady_clock::now()
+                                   .time_since_epoch()
+                                   .count();
+        v ^= (unsigned long long)reinterpret_cast<uintptr_t>(&ctr) * 0x9E3779B97F4A7C15ull;
+        return v | 1ull;
+    }();
+    return seed + 0x9E3779B97F4A7C15ull * (ctr.fetch_add(1) + 1);
+}
+
+int dt_tiles_per_channel(const Geom& g)
+{
+    const int bpt = dt_nt_for(g.w) / g.nw;
+    return (int)((g.bands + bpt - 1) / bpt);
+}
+
+long long tc_dt_partials_impl(const Geom& g)
+{
+    const long long tiles = (long long)g.C * dt_tiles_per_channel(g);
+    return g.C + (tiles < kDtMaxGrid ? tiles : kDtMaxGrid) - 1;
 }
 
 template <int WS>
-cudaError_t dt_launch_ws(const Geom& g, const void* x, const void* dy, float* partials,
-                         const Launch& L)
+cudaError_t dt_launch_ws(const Geom& g, const void* x, const void* dy, float* workspace,
+                         float* dT, bool after_dx, const Launch& L)
 {
     using F = DtCfg<WS>;
     const DtLayout lay = dt_layout<WS>();
@@ -533,14 +634,23 @@ cudaError_t dt_launch_ws(const Geom& g, const void* x, const void* dy, float* pa
     TcDtParams P;
     P.x = static_cast<const uint16_t*>(x);
     P.dy = static_cast<const uint16_t*>(dy);
-    P.partials = partials;
+    P.partials = workspace;
+    P.flags = reinterpret_cast<unsigned long long*>(workspace + dt_flags_offset(g));
+    P.token = next_launch_token();
+    P.dT = dT;
     P.C = g.C; P.H = g.H; P.W = g.W; P.nh = g.nh; P.nw = g.nw;
     P.bpt = F::NT / g.nw;
     P.bands = (int)g.bands;
     P.tpc = (P.bands + P.bpt - 1) / P.bpt;
-    P.ch = chunk_tiles(P.tpc);
-    P.chunks = (P.tpc + P.ch - 1) / P.ch;
-    P.items = g.C * P.chunks;
+    const int tiles = g.C * P.tpc;
+    int grid = L.num_sms < kDtMaxGrid ? L.num_sms : kDtMaxGrid;
+    if (grid > tiles)
+        grid = tiles;
+    if (grid < 1)
+        return cudaSuccess;
+    P.rq = tiles / grid;
+    P.rr = tiles - P.rq * grid;
+    P.dep_wait = after_dx ? 0 : 1;
     P.use_tmap = 0;
     P.kimg = 0;
     if (P.bpt % g.nh == 0) {
@@ -554,11 +664,6 @@ cudaError_t dt_launch_ws(const Geom& g, const void* x, const void* dy, float* pa
     P.off_woff = lay.off_woff; P.off_bar = lay.off_bar;
     P.budget = L.budget;
     P.status = L.status;
-    int grid = L.num_sms;
-    if (grid > P.items)
-        grid = P.items;
-    if (grid < 1)
-        return cudaSuccess;
     cudaError_t e = launch_pdl(wbmm_tc_dt_kernel<WS>, dim3(grid), dim3(kDtThreads), lay.total,
                                L.stream, P);
     if (e != cudaSuccess)
@@ -582,33 +687,36 @@ bool tc_dt_supported(const Geom& g)
     return true;
 }
 
-int tc_dt_chunks(const Geom& g)
+long long tc_dt_partials(const Geom& g)
 {
-    const int bpt = dt_nt_for(g.w) / g.nw;
-    const int tpc = (int)((g.bands + bpt - 1) / bpt);
-    const int ch = chunk_tiles(tpc);
-    return (tpc + ch - 1) / ch;
+    return tc_dt_partials_impl(g);
 }
 
-cudaError_t tc_dt_launch(const Geom& g, const void* x, const void* dy, float* partials,
-                         const Launch& L)
+long long tc_dt_workspace_floats(const Geom& g)
+{
+    // partial tables, then one 64-bit flag per table (8-byte aligned)
+    return dt_flags_offset(g) + 2 * tc_dt_partials(g);
+}
+
+cudaError_t tc_dt_launch(const Geom& g, const void* x, const void* dy, float* partials, float* dT,
+                         bool after_dx, const Launch& L)
 {
     switch (g.w) {
-    case 2: return dt_launch_ws<2>(g, x, dy, partials, L);
-    case 3: return dt_launch_ws<3>(g, x, dy, partials, L);
-    case 4: return dt_launch_ws<4>(g, x, dy, partials, L);
-    case 5: return dt_launch_ws<5>(g, x, dy, partials, L);
-    case 6: return dt_launch_ws<6>(g, x, dy, partials, L);
-    case 7: return dt_launch_ws<7>(g, x, dy, partials, L);
-    case 8: return dt_launch_ws<8>(g, x, dy, partials, L);
-    case 9: return dt_launch_ws<9>(g, x, dy, partials, L);
-    case 10: return dt_launch_ws<10>(g, x, dy, partials, L);
-    case 11: return dt_launch_ws<11>(g, x, dy, partials, L);
-    case 12: return dt_launch_ws<12>(g, x, dy, partials, L);
-    case 13: return dt_launch_ws<13>(g, x, dy, partials, L);
-    case 14: return dt_launch_ws<14>(g, x, dy, partials, L);
-    case 15: return dt_launch_ws<15>(g, x, dy, partials, L);
-    case 16: return dt_launch_ws<16>(g, x, dy, partials, L);
+    case 2: return dt_launch_ws<2>(g, x, dy, partials, dT, after_dx, L);
+    case 3: return dt_launch_ws<3>(g, x, dy, partials, dT, after_dx, L);
+    case 4: return dt_launch_ws<4>(g, x, dy, partials, dT, after_dx, L);
+    case 5: return dt_launch_ws<5>(g, x, dy, partials, dT, after_dx, L);
+    case 6: return dt_launch_ws<6>(g, x, dy, partials, dT, after_dx, L);
+    case 7: return dt_launch_ws<7>(g, x, dy, partials, dT, after_dx, L);
+    case 8: return dt_launch_ws<8>(g, x, dy, partials, dT, after_dx, L);
+    case 9: return dt_launch_ws<9>(g, x, dy, partials, dT, after_dx, L);
+    case 10: return dt_launch_ws<10>(g, x, dy, partials, dT, after_dx, L);
+    case 11: return dt_launch_ws<11>(g, x, dy, partials, dT, after_dx, L);
+    case 12: return dt_launch_ws<12>(g, x, dy, partials, dT, after_dx, L);
+    case 13: return dt_launch_ws<13>(g, x, dy, partials, dT, after_dx, L);
+    case 14: return dt_launch_ws<14>(g, x, dy, partials, dT, after_dx, L);
+    case 15: return dt_launch_ws<15>(g, x, dy, partials, dT, after_dx, L);
+    case 16: return dt_launch_ws<16>(g, x, dy, partials, dT, after_dx, L);
     default: return cudaErrorInvalidValue;
     }
 }
