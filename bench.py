@@ -89,6 +89,7 @@ def kernel_bytes(wl, name):
     return {"forward": 2 * m + tbl, "backward_dx": 2 * m + tbl,
             "backward_dt": 2 * m + wl.C * wl.t * 4,
             "forward_cached": 2 * m + wl.C * wl.d * wl.d * e,
+            "forward_cached_dw3x3": 2 * m + wl.C * wl.d * wl.d * e + wl.C * 9 * e,
             "dw3x3": 2 * m + wl.C * 9 * e}[name]
 
 
@@ -96,6 +97,8 @@ def kernel_flops(wl, name):
     n = wl.B * wl.C * wl.H * wl.W
     if name == "dw3x3":
         return 18.0 * n
+    if name == "forward_cached_dw3x3":
+        return 2.0 * n * wl.d + 18.0 * n
     return 2.0 * n * wl.d
 
 
@@ -198,6 +201,12 @@ class Arm:
             return ["forward_cached", "dw3x3"]
         return ["forward"]
 
+    def alternatives(self):
+        """Other launches of the same step, timed for reference only: the
+        fused cached forward + 3x3 (one launch; slower on 224x224 planes,
+        where its stencil work blocks the epilogue warps)."""
+        return ["forward_cached_dw3x3"] if self.wl.kind == "cached_dw" else []
+
     def calls(self):
         """The step as a user issues it: the training step is one forward
         and one backward call that returns both dX and dT."""
@@ -217,6 +226,8 @@ class Arm:
             wb.wbmm_backward(s["x"], self.T, s["dY"], s["dX"], self.dT, self.ws, w)
         elif name == "forward_cached":
             wb.wbmm_forward_cached(s["x"], self.M, None, s["y"], w)
+        elif name == "forward_cached_dw3x3":
+            wb.wbmm_forward_cached(s["x"], self.M, self.K, s["z"], w)
         elif name == "dw3x3":
             wb.wbmm_dw3x3(s["y"], self.K, s["z"])
 
@@ -364,6 +375,21 @@ def run_gpu(args, rank, world, local_rank):
             evs[k][j][1].record(stream)
     torch.cuda.synchronize()
     barrier(world)
+    alt = {}
+    for name in wb_arm.alternatives():
+        s = wb_arm.sets[0]
+        for _ in range(3):
+            wb_arm.launch(name, s)
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        a0.record(stream)
+        for k in range(K):
+            wb_arm.launch(name, wb_arm.sets[k % len(wb_arm.sets)])
+        a1.record(stream)
+        torch.cuda.synchronize()
+        us = max_over_ranks(a0.elapsed_time(a1) / K, world, dev) * 1e3
+        alt[name] = {"us": round(us, 2),
+                     "gbs": round(kernel_bytes(wl, name) / (us * 1e-6) / 1e9, 1)}
     kern = {}
     for j, name in enumerate(names):
         avg = sum(evs[k][j][0].elapsed_time(evs[k][j][1]) for k in range(K)) / K
@@ -423,7 +449,7 @@ def run_gpu(args, rank, world, local_rank):
             "workload": "%s: B%d C%d %dx%d w%d (%s)" % (wl.name, wl.B, wl.C, wl.H, wl.W, wl.w,
                                                       {"train": "forward + dX + dT",
                                                        "forward": "forward",
-                                                       "cached_dw": "cached forward + 3x3"}[wl.kind]),
+                                                       "cached_dw": "cached forward, then 3x3"}[wl.kind]),
             "B": wl.B, "C_per_gpu": wl.C, "H": wl.H, "W": wl.W, "w": wl.w,
             "parallelism": "channel-sharded, %d rank(s), no collective" % world,
             "channels_of_rank0": list(channel_range(wl.C * world, world, 0)),
@@ -452,6 +478,8 @@ def run_gpu(args, rank, world, local_rank):
                               "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                               "frac": round(kern[dom]["tflops"] / peaks["bf16_tflops"], 4),
                               "traffic": None, "peak_source": peaks["source"]}
+    if alt:
+        result["alternatives"] = alt
     step_roof_tf = min(peaks["bf16_tflops"], step_flops(wl) / step_bytes(wl) * peaks["hbm_gbs"] / 1e3)
     result["step_roofline_frac"] = round(value / world / step_roof_tf, 4)
     result["e2e"] = {"value": round(flops_all / (e2e_ms * 1e-3) / 1e12, 4), "unit": "TFLOP/s",

@@ -124,8 +124,12 @@ WBMM_API wbmm_status wbmm_cache_matrices(const void *T, void *M, int C, int w,
  *       y is rounded to dt exactly as a separate wbmm_forward_cached call
  *       would store it, so the fused result equals the two-call result.
  *   x [B,C,H,W], M [C,d,d], dw3x3 [C,1,3,3] or NULL, out [B,C,H,W]; dtype dt.
- * Errors: as wbmm_forward; UNSUPPORTED when the fused path's per-plane
- * buffer (H*W elements) exceeds its limit.
+ * Errors: as wbmm_forward; UNSUPPORTED for a fused call the fused kernel
+ * does not cover: fp32 maps, W not a multiple of 8, a tile of window rows
+ * that does not divide the image's window rows (the kernel processes whole
+ * image planes), or a plane of H*W bf16 elements beyond the per-SM buffer
+ * (about 100 KB beside the pipeline at w = 14).  out must not overlap x, M or
+ * dw3x3.
  */
 WBMM_API wbmm_status wbmm_forward_cached(const void *x, const void *M, const void *dw3x3,
                                 void *out, int B, int C, int H, int W, int w,

@@ -150,6 +150,54 @@ def test_forward_cached_bf16(shape):
     check_bf16(to_np(y2), ref, bound, "cached random M")
 
 
+# (B, C, H, W, w): fused work units of one tile holding several planes
+# (56x56, 48x48 at w=16) and of one plane spanning several tiles (112x56 at
+# w=7, 224x224)
+FUSED_SHAPES = [(3, 2, 56, 56, 14), (2, 3, 112, 56, 7), (2, 2, 48, 48, 16), (2, 3, 224, 224, 14)]
+
+
+@pytest.mark.parametrize("shape", FUSED_SHAPES, ids=lambda s: "x".join(map(str, s)))
+def test_fused_cached_dw3x3_matches_two_calls(shape):
+    B, C, H, W, w = shape
+    x = gen((B, C, H, W), 21)
+    T = gen((C, (2 * w - 1) ** 2), 22, scale=0.02)
+    K = gen((C, 1, 3, 3), 23, scale=1.0 / 3.0)
+    M = wb.cache_matrices(T, w)
+    z = wb.forward_cached(x, M, w, dw=K)
+    torch.cuda.synchronize()
+    assert wb.wbmm_get_device_status() == 0
+    assert wb.wbmm_last_path() == 1
+    y = wb.forward_cached(x, M, w)
+    z2 = wb.dw3x3(y, K)
+    torch.cuda.synchronize()
+    # y rounded to bf16 between the stages in both paths: the same bits
+    assert torch.equal(z, z2)
+    if H * W >= 224 * 224:
+        # and within tolerance of the oracle's 3x3 of the oracle's y
+        yr, Kr = to_np(y), to_np(K)
+        ref = oracle.dw3x3(oracle.forward(to_np(x), to_np(T), w), Kr)
+        bound = oracle.dw3x3(forward_rowbound(to_np(x), to_np(T), w), np.abs(Kr))
+        check_bf16(to_np(z), ref, bound, "fused cached + 3x3")
+
+
+def test_fused_cached_dw3x3_unsupported_shapes():
+    # window rows per tile (16) and per image (3) do not divide each other
+    x = gen((2, 2, 42, 56), 24)
+    M = wb.cache_matrices(gen((2, 729), 25, scale=0.02), 14)
+    K = gen((2, 1, 3, 3), 26)
+    before = wb.wbmm_launch_count()
+    with pytest.raises(wb.WbmmError) as e:
+        wb.forward_cached(x, M, 14, dw=K)
+    assert e.value.status == 5
+    # fp32 maps
+    xf = gen((1, 2, 14, 14), 27, torch.float32)
+    Mf = wb.cache_matrices(gen((2, 169), 28, torch.float32, 0.02), 7)
+    with pytest.raises(wb.WbmmError) as e:
+        wb.forward_cached(xf, Mf, 7, dw=gen((2, 1, 3, 3), 29, torch.float32))
+    assert e.value.status == 5
+    assert wb.wbmm_launch_count() == before + 1     # only the fp32 cache_matrices
+
+
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 @pytest.mark.parametrize("hw", [(37, 70), (40, 64), (33, 8)])  # scalar and 16-byte-row paths
 def test_dw3x3(dtype, hw):

@@ -4,6 +4,7 @@
 // mixing and the bounded-wait self-test.
 #include <cuda_bf16.h>
 
+#include "dw_common.cuh"
 #include "ptx_sm100.cuh"
 #include "wbmm_internal.h"
 
@@ -246,37 +247,11 @@ __global__ void __launch_bounds__(256) dw3x3_bf16_vec_kernel(const uint16_t* __r
         const int h = h0 + rr;
         if (h >= H)
             continue;
-        float acc[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-            acc[j] = 0.0f;
-#pragma unroll
-        for (int a = 0; a < 3; ++a) {
-            const uint16_t* row = s16 + (long long)(rr + a) * W + 8 * v;
-            float vals[10];
-            vals[0] = v > 0 ? __bfloat162float(__ushort_as_bfloat16(row[-1])) : 0.0f;
-            const uint4 mid = sband[(rr + a) * nvec + v];
-            const uint32_t w4[4] = {mid.x, mid.y, mid.z, mid.w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                vals[1 + 2 * j] = __uint_as_float(w4[j] << 16);
-                vals[2 + 2 * j] = __uint_as_float(w4[j] & 0xFFFF0000u);
-            }
-            vals[9] = v + 1 < nvec ? __bfloat162float(__ushort_as_bfloat16(row[8])) : 0.0f;
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-#pragma unroll
-                for (int e = 0; e < 3; ++e)
-                    acc[j] = __fmaf_rn(k[a * 3 + e], vals[j + e], acc[j]);
-        }
-        uint32_t packed[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const uint32_t lo = __bfloat16_as_ushort(__float2bfloat16_rn(acc[2 * j]));
-            const uint32_t hi = __bfloat16_as_ushort(__float2bfloat16_rn(acc[2 * j + 1]));
-            packed[j] = lo | (hi << 16);
-        }
-        zp[(long long)h * nvec + v] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+        // halo rows outside the image were staged as zeros
+        const uint16_t* rows[3] = {s16 + (long long)rr * W + 8 * v,
+                                   s16 + (long long)(rr + 1) * W + 8 * v,
+                                   s16 + (long long)(rr + 2) * W + 8 * v};
+        zp[(long long)h * nvec + v] = dw3x3_row8(rows, v, nvec, k);
     }
 }
 

@@ -26,11 +26,19 @@
 //
 // Pipeline: raw ring (R slots) -> operand stages (2) -> accumulators (2)
 // -> output slots (2).
+//
+// Fused 3x3 (cached matrices only): the work is split in units of whole image
+// planes (one plane of several tiles, or one tile of several planes), the
+// epilogue writes bf16 y into a buffer for the unit that replaces the output
+// slots, and after the unit's last tile the epilogue warps apply the 3x3
+// mixing to each of its planes from shared memory (zero outside the plane)
+// and store z; y never reaches HBM.
 // Every wait is bounded; a wait that runs out raises the CTA's abort flag and
 // the device status word, and every role then runs its loop without doing
 // work so that all threads reach the drain and the TMEM release.
 #include <cuda_bf16.h>
 
+#include "dw_common.cuh"
 #include "ptx_sm100.cuh"
 #include "tc_common.cuh"
 #include "wbmm_internal.h"
@@ -81,6 +89,11 @@ struct TcFwdParams {
     uint32_t off_raw, off_b, off_out, off_tbl, off_woff, off_bar;
     unsigned long long budget;
     int* status;
+    int fused;              // 3x3 mixing applied to y in shared memory
+    int ub;                 // bands per work unit (fused: whole planes)
+    int tpp;                // tiles per work unit (fused), else 1
+    const uint16_t* dw;     // 3x3 weights [C][9] (fused)
+    uint16_t* z;            // mixed output map (fused)
 };
 
 struct Bars {
@@ -208,10 +221,12 @@ __global__ void __launch_bounds__(kThreads, 1) wbmm_tc_fwd_kernel(const __grid_c
     volatile int* abort = &S.abort;
     const int R = P.R;
 
-    // Contiguous, balanced range of items for this CTA.
-    const int q = P.items / (int)gridDim.x, rem = P.items % (int)gridDim.x;
-    const int it0 = (int)blockIdx.x * q + ((int)blockIdx.x < rem ? (int)blockIdx.x : rem);
-    const int n_it = q + ((int)blockIdx.x < rem ? 1 : 0);
+    // Contiguous, balanced range of items for this CTA, in units of tpp
+    // tiles (whole image planes when fused).
+    const int units = P.items / P.tpp;
+    const int q = units / (int)gridDim.x, rem = units % (int)gridDim.x;
+    const int it0 = ((int)blockIdx.x * q + ((int)blockIdx.x < rem ? (int)blockIdx.x : rem)) * P.tpp;
+    const int n_it = (q + ((int)blockIdx.x < rem ? 1 : 0)) * P.tpp;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kMaxRing; ++i) {
@@ -353,7 +368,8 @@ __global__ void __launch_bounds__(kThreads, 1) wbmm_tc_fwd_kernel(const __grid_c
         // ------------------------------------------------------ storer
         // Bulk-stores each finished output slot (one run per lane), waits
         // until the copies have read shared memory, then frees the slot.
-        for (int seq = 0; seq < n_it; ++seq) {
+        // Idle when fused: the epilogue warps write z themselves.
+        for (int seq = 0; seq < (P.fused ? 0 : n_it); ++seq) {
             const int os = seq & 1;
             bool ok = !*abort;
             ok = ok && mbar_wait(&S.out_full[os], (seq >> 1) & 1, abort, P.budget, P.status);
@@ -456,12 +472,14 @@ __global__ void __launch_bounds__(kThreads, 1) wbmm_tc_fwd_kernel(const __grid_c
             const int ab = seq & 1, os = seq & 1;
             bool ok = !*abort;
             ok = ok && mbar_wait(&S.acc_full[ab], (seq >> 1) & 1, abort, P.budget, P.status);
-            if (seq >= 2)
+            if (seq >= 2 && !P.fused)
                 ok = ok && mbar_wait(&S.out_empty[os], ((seq >> 1) - 1) & 1, abort, P.budget,
                                      P.status);
             ok = __all_sync(0xffffffffu, ok);
             tc_fence_after();
-            uint16_t* out = reinterpret_cast<uint16_t*>(out_base + (size_t)os * F::RAW_BYTES);
+            uint16_t* out = P.fused
+                ? reinterpret_cast<uint16_t*>(out_base) + (long long)(t.band0 % P.ub) * WS * P.W
+                : reinterpret_cast<uint16_t*>(out_base + (size_t)os * F::RAW_BYTES);
             if (ok) {
                 const uint32_t lrow = tmem + ((uint32_t)(quarter * 32) << 16) + F::D_COL0 +
                                       (uint32_t)(ab * F::MT * F::NT);
@@ -514,7 +532,34 @@ __global__ void __launch_bounds__(kThreads, 1) wbmm_tc_fwd_kernel(const __grid_c
             __syncwarp();
             if (ok && lane == 0) {
                 mbar_arrive(&S.acc_empty[ab]);
-                mbar_arrive(&S.out_full[os]);
+                if (!P.fused)
+                    mbar_arrive(&S.out_full[os]);
+            }
+            if (P.fused && (seq + 1) % P.tpp == 0) {
+                // the unit's last tile: y of its planes is complete in shared memory
+                named_bar_sync(4, kEpiWarps * 32);
+                const int et = threadIdx.x - kEpiWarp0 * 32;
+                const int ub0 = t.band0 - t.band0 % P.ub;
+                const int left = P.bands - ub0;
+                const int planes = (left < P.ub ? left : P.ub) / P.nh;
+                const int b0 = ub0 / P.nh;
+                float kw[9];
+#pragma unroll
+                for (int m = 0; m < 9; ++m)
+                    kw[m] = __bfloat162float(__ushort_as_bfloat16(P.dw[t.c * 9 + m]));
+                const int nvec = P.W / 8, per_plane = P.H * nvec;
+                for (int o = et; o < planes * per_plane; o += kEpiWarps * 32) {
+                    const int j = o / per_plane, r = o - j * per_plane;
+                    const int h = r / nvec, v = r - (r / nvec) * nvec;
+                    const uint16_t* mid = reinterpret_cast<const uint16_t*>(out_base) +
+                                          ((long long)j * P.H + h) * P.W + 8 * v;
+                    const uint16_t* rows[3] = {h > 0 ? mid - P.W : nullptr, mid,
+                                               h + 1 < P.H ? mid + P.W : nullptr};
+                    uint4* zp = reinterpret_cast<uint4*>(
+                        P.z + (((long long)(b0 + j) * P.C + t.c) * P.H) * P.W);
+                    zp[r] = dw3x3_row8(rows, v, nvec, kw);
+                }
+                named_bar_sync(4, kEpiWarps * 32);   // read before the buffer is rewritten
             }
         }
     }
@@ -541,13 +586,20 @@ struct FwdLayout {
     int R;
 };
 
+// out_bytes: the output region, two band slots, or one image plane when the
+// 3x3 mixing is fused.
 template <int WS>
-FwdLayout fwd_layout()
+FwdLayout fwd_layout(uint32_t out_bytes)
 {
     using F = FwdCfg<WS>;
     FwdLayout L;
-    const uint32_t fixed = 2 * F::B_BYTES + 2 * F::RAW_BYTES + 2 * F::TCOPY_BYTES + F::NT * 4 +
+    const uint32_t fixed = 2 * F::B_BYTES + out_bytes + 2 * F::TCOPY_BYTES + F::NT * 4 +
                            align_up(sizeof(Bars), 16) + 3 * 1024;
+    if (fixed >= kSmemMax) {
+        L.R = 0;
+        L.total = kSmemMax + 1;
+        return L;
+    }
     int R = (int)((kSmemMax - fixed) / F::RAW_BYTES);
     if (R > kMaxRing)
         R = kMaxRing;
@@ -558,7 +610,7 @@ FwdLayout fwd_layout()
     L.off_raw = align_up(off, 128);
     off = L.off_raw + (uint32_t)R * F::RAW_BYTES;
     L.off_out = align_up(off, 128);
-    off = L.off_out + 2 * F::RAW_BYTES;
+    off = L.off_out + out_bytes;
     L.off_tbl = align_up(off, 16);
     off = L.off_tbl + 2 * F::TCOPY_BYTES;
     L.off_woff = align_up(off, 16);
@@ -573,23 +625,46 @@ FwdLayout fwd_layout()
     return L;
 }
 
+// Bands per fused work unit: one plane of several tiles or one tile of
+// several planes; 0 when neither divides the other.
+int fused_unit_bands(const Geom& g, int bpt)
+{
+    if (g.nh % bpt == 0)
+        return g.nh;
+    if (bpt % g.nh == 0)
+        return bpt;
+    return 0;
+}
+
+template <int WS>
+uint32_t out_region_bytes(const Geom& g, bool fused)
+{
+    if (!fused)
+        return 2 * FwdCfg<WS>::RAW_BYTES;
+    const int ub = fused_unit_bands(g, FwdCfg<WS>::NT / g.nw);
+    return align_up((uint32_t)((long long)ub * WS * g.W * 2), 128);
+}
+
+// y: the output map (z when fused); dw: the 3x3 weights when fused, else null.
 template <int WS, int MODE>
-cudaError_t launch_ws(const Geom& g, const void* x, const void* src, void* y, const Launch& L)
+cudaError_t launch_ws(const Geom& g, const void* x, const void* src, void* y, const void* dw,
+                      const Launch& L)
 {
     using F = FwdCfg<WS>;
-    const FwdLayout lay = fwd_layout<WS>();
+    const bool fused = dw != nullptr;
+    const FwdLayout lay = fwd_layout<WS>(out_region_bytes<WS>(g, fused));
     if (lay.R < 2 || lay.total > kSmemMax)
         return cudaErrorInvalidConfiguration;
-    static unsigned long long configured = 0;
+    static int configured_smem[64] = {0};
     int dev = 0;
     cudaGetDevice(&dev);
-    if (!(configured & (1ull << (dev & 63)))) {
+    if (configured_smem[dev & 63] < (int)kSmemMax) {
         cudaError_t e = cudaFuncSetAttribute(wbmm_tc_fwd_kernel<WS, MODE>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)lay.total);
+                                             (int)kSmemMax);
         if (e != cudaSuccess)
             return e;
-        configured |= 1ull << (dev & 63);
+        configured_smem[dev & 63] = (int)kSmemMax;
     }
     TcFwdParams P;
     P.x = static_cast<const uint16_t*>(x);
@@ -601,6 +676,11 @@ cudaError_t launch_ws(const Geom& g, const void* x, const void* src, void* y, co
     P.tpc = (P.bands + P.bpt - 1) / P.bpt;
     P.items = g.C * P.tpc;
     P.R = lay.R;
+    P.fused = fused ? 1 : 0;
+    P.ub = fused ? fused_unit_bands(g, P.bpt) : P.bpt;
+    P.tpp = fused ? P.ub / P.bpt : 1;
+    P.dw = static_cast<const uint16_t*>(dw);
+    P.z = fused ? static_cast<uint16_t*>(y) : nullptr;
     P.use_tmap = 0;
     P.kimg = 0;
     if (P.bpt % g.nh == 0) {
@@ -615,8 +695,8 @@ cudaError_t launch_ws(const Geom& g, const void* x, const void* src, void* y, co
     P.budget = L.budget;
     P.status = L.status;
     int grid = L.num_sms;
-    if (grid > P.items)
-        grid = P.items;
+    if (grid > P.items / P.tpp)
+        grid = P.items / P.tpp;
     if (grid < 1)
         return cudaSuccess;
     cudaError_t e = launch_pdl(wbmm_tc_fwd_kernel<WS, MODE>, dim3(grid), dim3(kThreads),
@@ -629,13 +709,20 @@ cudaError_t launch_ws(const Geom& g, const void* x, const void* src, void* y, co
 
 template <int WS>
 cudaError_t launch_mode(const Geom& g, AMode mode, const void* x, const void* src, void* y,
-                        const Launch& L)
+                        const void* dw, const Launch& L)
 {
     switch (mode) {
-    case kTable: return launch_ws<WS, kTable>(g, x, src, y, L);
-    case kTableFlip: return launch_ws<WS, kTableFlip>(g, x, src, y, L);
-    default: return launch_ws<WS, kCached>(g, x, src, y, L);
+    case kTable: return launch_ws<WS, kTable>(g, x, src, y, nullptr, L);
+    case kTableFlip: return launch_ws<WS, kTableFlip>(g, x, src, y, nullptr, L);
+    default: return launch_ws<WS, kCached>(g, x, src, y, dw, L);
     }
+}
+
+template <int WS>
+bool fused_fits(const Geom& g)
+{
+    const FwdLayout lay = fwd_layout<WS>(out_region_bytes<WS>(g, true));
+    return lay.R >= 2 && lay.total <= kSmemMax;
 }
 
 int nt_for(int w)
@@ -648,8 +735,6 @@ int nt_for(int w)
 
 bool tc_fwd_supported(const Geom& g, bool fused)
 {
-    if (fused)
-        return false;
     if (g.w < 2 || g.w > 16)
         return false;
     if (g.nw > nt_for(g.w))
@@ -660,29 +745,51 @@ bool tc_fwd_supported(const Geom& g, bool fused)
     // 32-bit tile bookkeeping
     if (g.bands * (long long)g.C >= (1ll << 31))
         return false;
+    if (fused) {
+        // tiles are whole bands of one plane, planes whole 16-byte rows, and
+        // one plane of y fits in shared memory beside the pipeline
+        if (g.W % 8 != 0 || fused_unit_bands(g, nt_for(g.w) / g.nw) == 0)
+            return false;
+        switch (g.w) {
+        case 2: return fused_fits<2>(g);
+        case 3: return fused_fits<3>(g);
+        case 4: return fused_fits<4>(g);
+        case 5: return fused_fits<5>(g);
+        case 6: return fused_fits<6>(g);
+        case 7: return fused_fits<7>(g);
+        case 8: return fused_fits<8>(g);
+        case 9: return fused_fits<9>(g);
+        case 10: return fused_fits<10>(g);
+        case 11: return fused_fits<11>(g);
+        case 12: return fused_fits<12>(g);
+        case 13: return fused_fits<13>(g);
+        case 14: return fused_fits<14>(g);
+        case 15: return fused_fits<15>(g);
+        default: return fused_fits<16>(g);
+        }
+    }
     return true;
 }
 
 cudaError_t tc_fwd_launch(const Geom& g, AMode mode, const void* x, const void* src, void* y,
                           const void* dw, const Launch& L)
 {
-    (void)dw;
     switch (g.w) {
-    case 2: return launch_mode<2>(g, mode, x, src, y, L);
-    case 3: return launch_mode<3>(g, mode, x, src, y, L);
-    case 4: return launch_mode<4>(g, mode, x, src, y, L);
-    case 5: return launch_mode<5>(g, mode, x, src, y, L);
-    case 6: return launch_mode<6>(g, mode, x, src, y, L);
-    case 7: return launch_mode<7>(g, mode, x, src, y, L);
-    case 8: return launch_mode<8>(g, mode, x, src, y, L);
-    case 9: return launch_mode<9>(g, mode, x, src, y, L);
-    case 10: return launch_mode<10>(g, mode, x, src, y, L);
-    case 11: return launch_mode<11>(g, mode, x, src, y, L);
-    case 12: return launch_mode<12>(g, mode, x, src, y, L);
-    case 13: return launch_mode<13>(g, mode, x, src, y, L);
-    case 14: return launch_mode<14>(g, mode, x, src, y, L);
-    case 15: return launch_mode<15>(g, mode, x, src, y, L);
-    case 16: return launch_mode<16>(g, mode, x, src, y, L);
+    case 2: return launch_mode<2>(g, mode, x, src, y, dw, L);
+    case 3: return launch_mode<3>(g, mode, x, src, y, dw, L);
+    case 4: return launch_mode<4>(g, mode, x, src, y, dw, L);
+    case 5: return launch_mode<5>(g, mode, x, src, y, dw, L);
+    case 6: return launch_mode<6>(g, mode, x, src, y, dw, L);
+    case 7: return launch_mode<7>(g, mode, x, src, y, dw, L);
+    case 8: return launch_mode<8>(g, mode, x, src, y, dw, L);
+    case 9: return launch_mode<9>(g, mode, x, src, y, dw, L);
+    case 10: return launch_mode<10>(g, mode, x, src, y, dw, L);
+    case 11: return launch_mode<11>(g, mode, x, src, y, dw, L);
+    case 12: return launch_mode<12>(g, mode, x, src, y, dw, L);
+    case 13: return launch_mode<13>(g, mode, x, src, y, dw, L);
+    case 14: return launch_mode<14>(g, mode, x, src, y, dw, L);
+    case 15: return launch_mode<15>(g, mode, x, src, y, dw, L);
+    case 16: return launch_mode<16>(g, mode, x, src, y, dw, L);
     default: return cudaErrorInvalidValue;
     }
 }
