@@ -38,11 +38,19 @@ L2_BYTES = 126 * 2 ** 20
 WORKLOADS = {
     "train": "train_bf16",
     "fwd": "fwd_bf16",
+    "fwd32": "fwd_f32",
     "sweep7": "sweep_w7",
     "sweep14": "sweep_w14",
     "sweep28": "sweep_w28",
     "cached": "hires_cached_dw",
 }
+
+
+def fp32_fma_peak_tflops(dev):
+    """CUDA-core fp32 peak: 128 fp32 lanes per SM, one FMA (2 FLOP) per lane
+    per cycle, at the B200's 1965 MHz maximum SM clock."""
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    return sms * 128 * 2 * 1.965e9 / 1e12
 
 
 def load_peaks():
@@ -83,7 +91,7 @@ def step_bytes(wl):
 
 
 def kernel_bytes(wl, name):
-    e = 2
+    e = 2 if wl.dtype == "bf16" else 4
     m = wl.B * wl.C * wl.H * wl.W * e
     tbl = wl.C * wl.t * e
     return {"forward": 2 * m + tbl, "backward_dx": 2 * m + tbl,
@@ -443,7 +451,7 @@ def run_gpu(args, rank, world, local_rank):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16",
+        "dtype": wl.dtype,
         "data": "synthetic",
         "config": {
             "workload": "%s: B%d C%d %dx%d w%d (%s)" % (wl.name, wl.B, wl.C, wl.H, wl.W, wl.w,
@@ -467,7 +475,14 @@ def run_gpu(args, rank, world, local_rank):
     dom = max(kern, key=lambda n: kern[n]["us"])
     ai = kernel_flops(wl, dom) / kernel_bytes(wl, dom)
     ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
-    if ai < ridge:
+    alu_tf = fp32_fma_peak_tflops(dev)
+    if wl.dtype == "f32" and ai >= alu_tf * 1e12 / (peaks["hbm_gbs"] * 1e9):
+        # fp32 runs on the CUDA cores: bound by their FMA rate
+        result["roofline"] = {"bound": "alu", "kernel": dom, "achieved": kern[dom]["tflops"],
+                              "peak": round(alu_tf, 1), "unit": "TFLOP/s",
+                              "frac": round(kern[dom]["tflops"] / alu_tf, 4), "traffic": None,
+                              "peak_source": "derived: SMs x 128 fp32 lanes x 2 FLOP x 1965 MHz"}
+    elif ai < ridge:
         result["roofline"] = {"bound": "hbm", "kernel": dom, "achieved": kern[dom]["gbs"],
                               "peak": peaks["hbm_gbs"], "unit": "GB/s",
                               "frac": round(kern[dom]["gbs"] / peaks["hbm_gbs"], 4),
@@ -480,7 +495,8 @@ def run_gpu(args, rank, world, local_rank):
                               "traffic": None, "peak_source": peaks["source"]}
     if alt:
         result["alternatives"] = alt
-    step_roof_tf = min(peaks["bf16_tflops"], step_flops(wl) / step_bytes(wl) * peaks["hbm_gbs"] / 1e3)
+    top = alu_tf if wl.dtype == "f32" else peaks["bf16_tflops"]
+    step_roof_tf = min(top, step_flops(wl) / step_bytes(wl) * peaks["hbm_gbs"] / 1e3)
     result["step_roofline_frac"] = round(value / world / step_roof_tf, 4)
     result["e2e"] = {"value": round(flops_all / (e2e_ms * 1e-3) / 1e12, 4), "unit": "TFLOP/s",
                      "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d,

@@ -55,6 +55,7 @@ class Workload:
 WORKLOADS = {
     "tiny_fp32": Workload("tiny_fp32", 1, 4, 14, 14, 7, "f32", "normal", "forward"),
     "fwd_bf16": Workload("fwd_bf16", 64, 128, 56, 56, 14, "bf16", "truncated", "forward"),
+    "fwd_f32": Workload("fwd_f32", 64, 128, 56, 56, 14, "f32", "truncated", "forward"),
     "train_bf16": Workload("train_bf16", 128, 256, 28, 28, 14, "bf16", "truncated", "train"),
     "sweep_w7": Workload("sweep_w7", 32, 256, 112, 112, 7, "bf16", "normal", "forward"),
     "sweep_w14": Workload("sweep_w14", 32, 256, 112, 112, 14, "bf16", "normal", "forward"),

@@ -4,6 +4,8 @@
 // mixing and the bounded-wait self-test.
 #include <cuda_bf16.h>
 
+#include <utility>
+
 #include "dw_common.cuh"
 #include "ptx_sm100.cuh"
 #include "wbmm_internal.h"
@@ -69,6 +71,88 @@ __global__ void simt_fwd_kernel(const TIn* __restrict__ x, const TIn* __restrict
             }
         }
         yb[p * W + j * w + q] = from_f<TIn>(acc);
+    }
+}
+
+// ------------------------------------------------ forward, table modes
+// Register-tiled form of the same sums for the table modes and w <= 32: a
+// thread computes QC consecutive outputs (p, q0 .. q0+QC-1) of one window.
+// For each input row r it loads the QC + w - 1 table entries of row p - r
+// that those outputs use, then for each input s one x value feeds QC fused
+// multiply-adds with static indices; shared-memory loads per FMA drop from 2
+// to about 2/QC.  Each output is still one fp32 sum in (r, s) order, so the
+// result is bit-identical to simt_fwd_kernel.  A block takes `rb`
+// consecutive bands of one channel; the table (reversed end to end for the
+// input gradient) and the bands sit in shared memory as fp32.
+template <int WS>
+struct RowCfg {
+    static constexpr int QC = WS <= 16 ? WS : (WS + 1) / 2;   // outputs per thread
+    static constexpr int NQ = (WS + QC - 1) / QC;
+    static constexpr int L = 2 * WS - 1;
+    static constexpr int TSZ = L * L;
+    static constexpr int TPAD = (TSZ + QC + 3) / 4 * 4;        // table + overhang of the last chunk
+};
+
+template <typename TIn, int WS, bool FLIP>
+__global__ void __launch_bounds__(256) simt_fwd_rows_kernel(const TIn* __restrict__ x,
+                                                            const TIn* __restrict__ T,
+                                                            TIn* __restrict__ y, int C, int H,
+                                                            int W, int nh, int nw, int bands,
+                                                            int rb, int groups)
+{
+    using F = RowCfg<WS>;
+    extern __shared__ float sm[];
+    grid_dep_wait();
+    grid_dep_launch();
+    float* tbl = sm;
+    float* sb = sm + F::TPAD;
+    const int c = (int)(blockIdx.x / groups);
+    const int g0 = (int)(blockIdx.x - c * groups) * rb;
+    const int nb = bands - g0 < rb ? bands - g0 : rb;
+    for (int k = threadIdx.x; k < F::TPAD; k += blockDim.x)
+        tbl[k] = k < F::TSZ ? to_f(T[(long long)c * F::TSZ + (FLIP ? F::TSZ - 1 - k : k)]) : 0.0f;
+    const int band_elems = WS * W;
+    for (int e = threadIdx.x; e < nb * band_elems; e += blockDim.x) {
+        const int k = e / band_elems, off = e - k * band_elems;
+        const int g = g0 + k, b = g / nh, i = g - (g / nh) * nh;
+        sb[e] = to_f(x[(((long long)b * C + c) * H + (long long)i * WS) * W + off]);
+    }
+    __syncthreads();
+    const int items = nb * nw * F::NQ * WS;
+    for (int it = threadIdx.x; it < items; it += blockDim.x) {
+        const int p = it % WS;
+        int rest = it / WS;
+        const int qc = rest % F::NQ;
+        rest /= F::NQ;
+        const int j = rest % nw, k = rest / nw;
+        const int q0 = qc * F::QC;
+        const float* xw = sb + k * band_elems + j * WS;
+        float acc[F::QC];
+#pragma unroll
+        for (int qq = 0; qq < F::QC; ++qq)
+            acc[qq] = 0.0f;
+#pragma unroll 1
+        for (int r = 0; r < WS; ++r) {
+            const float* trow = tbl + (p - r + WS - 1) * F::L + q0;
+            float tv[F::QC + WS - 1];
+#pragma unroll
+            for (int m = 0; m < F::QC + WS - 1; ++m)
+                tv[m] = trow[m];
+            const float* xr = xw + r * W;
+#pragma unroll
+            for (int s2 = 0; s2 < WS; ++s2) {
+                const float xv = xr[s2];
+#pragma unroll
+                for (int qq = 0; qq < F::QC; ++qq)
+                    acc[qq] = __fmaf_rn(tv[qq - s2 + WS - 1], xv, acc[qq]);
+            }
+        }
+        const int g = g0 + k, b = g / nh, i = g - (g / nh) * nh;
+        TIn* yr = y + (((long long)b * C + c) * H + (long long)i * WS + p) * W + j * WS + q0;
+#pragma unroll
+        for (int qq = 0; qq < F::QC; ++qq)
+            if (q0 + qq < WS)
+                yr[qq] = from_f<TIn>(acc[qq]);
     }
 }
 
@@ -293,9 +377,70 @@ int simt_dt_chunks(const Geom& g)
     return (int)((g.bands + kSimtChunkBands - 1) / kSimtChunkBands);
 }
 
+namespace {
+
+template <typename E, int WS, bool FLIP>
+cudaError_t rows_launch_t(const Geom& g, const void* x, const void* T, void* y, const Launch& L)
+{
+    using F = RowCfg<WS>;
+    const size_t band_bytes = (size_t)WS * g.W * 4;
+    int rb = (int)((96 * 1024) / band_bytes);
+    if (rb > 4)
+        rb = 4;
+    if (rb < 1)
+        return cudaErrorInvalidConfiguration;
+    const size_t smem = (size_t)F::TPAD * 4 + (size_t)rb * band_bytes;
+    const int bands = (int)g.bands;
+    const int groups = (bands + rb - 1) / rb;
+    const long long blocks = (long long)g.C * groups;
+    if (blocks == 0)
+        return cudaSuccess;
+    if (blocks > 0x7fffffffLL)
+        return cudaErrorInvalidConfiguration;
+    cudaError_t e = set_smem(simt_fwd_rows_kernel<E, WS, FLIP>, smem);
+    if (e == cudaSuccess)
+        e = launch_pdl(simt_fwd_rows_kernel<E, WS, FLIP>, dim3((unsigned)blocks), dim3(256), smem,
+                       L.stream, static_cast<const E*>(x), static_cast<const E*>(T),
+                       static_cast<E*>(y), g.C, g.H, g.W, g.nh, g.nw, bands, rb, groups);
+    if (e != cudaSuccess)
+        return e;
+    note_launches(1);
+    return cudaGetLastError();
+}
+
+template <int WS>
+cudaError_t rows_launch_w(const Geom& g, bool flip, bool is_bf16, const void* x, const void* T,
+                          void* y, const Launch& L)
+{
+    if (is_bf16)
+        return flip ? rows_launch_t<__nv_bfloat16, WS, true>(g, x, T, y, L)
+                    : rows_launch_t<__nv_bfloat16, WS, false>(g, x, T, y, L);
+    return flip ? rows_launch_t<float, WS, true>(g, x, T, y, L)
+                : rows_launch_t<float, WS, false>(g, x, T, y, L);
+}
+
+// w = Is + 1 for Is = 0 .. 31
+template <int... Is>
+cudaError_t rows_dispatch(std::integer_sequence<int, Is...>, const Geom& g, bool flip,
+                          bool is_bf16, const void* x, const void* T, void* y, const Launch& L)
+{
+    cudaError_t e = cudaErrorInvalidValue;
+    ((g.w == Is + 1 ? (e = rows_launch_w<Is + 1>(g, flip, is_bf16, x, T, y, L), true) : false) ||
+     ...);
+    return e;
+}
+
+}  // namespace
+
 cudaError_t simt_fwd_launch(const Geom& g, AMode mode, bool is_bf16, const void* x,
                             const void* src, void* y, const Launch& L)
 {
+    if (mode != kCached && g.w >= 1 && g.w <= 32 && (size_t)g.w * g.W * 4 <= 96 * 1024) {
+        cudaError_t e = rows_dispatch(std::make_integer_sequence<int, 32>{}, g, mode == kTableFlip,
+                                      is_bf16, x, src, y, L);
+        if (e != cudaErrorInvalidValue)
+            return e;
+    }
     const size_t smem = ((mode == kCached ? 0 : (size_t)g.tsz) + (size_t)g.w * g.W) * 4;
     if (smem > kSimtSmemMax)
         return cudaErrorInvalidConfiguration;
