@@ -1,7 +1,8 @@
 // Tensor-core (tcgen05) WBMM forward and input-gradient kernel, window-major.
 //
-// The windows of a tile are the GEMM's M dimension and the output positions
-// of a window its N dimension:
+// The windows of a tile (128, or 256 as two M tiles when a window has at most
+// 64 padded positions) are the GEMM's M dimension and the output positions of
+// a window its N dimension:
 //
 //   D[n, (p, q)] = sum_{(r, s)} X[n, (r, s)] * M_c[(p, q), (r, s)]
 //
@@ -54,7 +55,11 @@ struct ToepCfg {
     static constexpr int NP = (WS * RP + 15) / 16 * 16;      // MMA N (output columns)
     static constexpr int QROWS = (WS - 1) * RP + NP;
     static constexpr int TSZ = (2 * WS - 1) * (2 * WS - 1);
-    static constexpr uint32_t A_BYTES = 128u * KP * 2;       // one operand stage
+    // 128-window M tiles per tile: two when a window is small (N <= 64), so
+    // that the per-tile fixed costs cover twice the data
+    static constexpr int MTW = NP <= 64 ? 2 : 1;
+    static constexpr int TW = 128 * MTW;                     // windows per tile
+    static constexpr uint32_t A_BYTES = (uint32_t)TW * KP * 2;   // one operand stage
     static constexpr uint32_t SBO_A = (uint32_t)KP * 16;     // bytes per 8-window group
     static constexpr uint32_t Q_BYTES = (uint32_t)QROWS * 32;
     static constexpr int LOADS = (NP + 31) / 32;             // 32-column TMEM loads per row
@@ -70,7 +75,6 @@ constexpr int kToepXformWarp0 = 3;
 constexpr int kToepEpiWarp0 = kToepXformWarp0 + kToepXformWarps;
 constexpr int kToepEpiWarps = 8;
 constexpr int kToepThreads = (kToepEpiWarp0 + kToepEpiWarps) * 32;
-constexpr int kToepTileWindows = 128;
 
 struct TcToepParams {
     TmapBytes map_x;        // input planes, one box = a half tile (use_tmap)
@@ -289,7 +293,7 @@ __global__ void __launch_bounds__(kToepThreads, 1)
         S.abort = 0;
         fence_mbar_init();
     }
-    for (int n = threadIdx.x; n < kToepTileWindows; n += kToepThreads) {
+    for (int n = threadIdx.x; n < F::TW; n += kToepThreads) {
         const int k = n / P.nw, j = n - k * P.nw;
         woff[n] = k * WS * P.W + j * WS;
     }
@@ -381,16 +385,22 @@ __global__ void __launch_bounds__(kToepThreads, 1)
                 tc_fence_after();
                 // K step k: operand columns [16k, 16k+16) and Q rows from
                 // (w - 1 - G*k)*RP: only the start-address fields move.
-                const uint64_t adesc0 =
-                    smem_desc(smem_u32(a_base + (size_t)st * F::A_BYTES), 128, F::SBO_A);
                 const uint64_t qdesc0 = smem_desc(
                     smem_u32(q_base + (size_t)qb * F::Q_BYTES) + (uint32_t)((WS - 1) * F::RP * 32),
                     128, 256);
-                const uint32_t d = tmem + (uint32_t)(ab * 256);
 #pragma unroll
-                for (int k = 0; k < F::KSTEPS; ++k)
-                    mma_ss(d, adesc0 + (uint64_t)(k * 16),
-                           qdesc0 - (uint64_t)(k * F::G * F::RP * 2), F::IDESC, k > 0 ? 1u : 0u);
+                for (int mt = 0; mt < F::MTW; ++mt) {
+                    // M tile mt: windows 128*mt .. (16 groups of 8 rows further)
+                    const uint64_t adesc0 = smem_desc(
+                        smem_u32(a_base + (size_t)st * F::A_BYTES) + (uint32_t)(mt * 16) * F::SBO_A,
+                        128, F::SBO_A);
+                    const uint32_t d = tmem + (uint32_t)(ab * 256 + mt * 128);
+#pragma unroll
+                    for (int k = 0; k < F::KSTEPS; ++k)
+                        mma_ss(d, adesc0 + (uint64_t)(k * 16),
+                               qdesc0 - (uint64_t)(k * F::G * F::RP * 2), F::IDESC,
+                               k > 0 ? 1u : 0u);
+                }
                 tc_commit(&S.acc_full[ab]);
             }
             // Drain: all issued MMAs complete before TMEM is released.
@@ -465,7 +475,6 @@ __global__ void __launch_bounds__(kToepThreads, 1)
         // other 32-column load, i.e. RL window rows of every window.
         const int quarter = warp & 3;
         const int hf = (warp - kToepEpiWarp0) >> 2;
-        const int n = quarter * 32 + lane;
         const int et = threadIdx.x - kToepEpiWarp0 * 32;
         const int c_first = toep_tile(P, it0).c;
         const int nch = toep_tile(P, it0 + n_it - 1).c - c_first + 1;
@@ -494,12 +503,15 @@ __global__ void __launch_bounds__(kToepThreads, 1)
             ok = ok && mbar_wait(&S.acc_full[ab], (seq >> 1) & 1, abort, P.budget, P.status);
             ok = __all_sync(0xffffffffu, ok);
             tc_fence_after();
-            if (ok && quarter * 32 < nwin) {
+#pragma unroll 1
+            for (int mt = 0; mt < F::MTW; ++mt) {
+              const int n = mt * 128 + quarter * 32 + lane;
+              if (ok && mt * 128 + quarter * 32 < nwin) {
                 const bool valid = n < nwin;
                 uint16_t* o0 = reinterpret_cast<uint16_t*>(a_base + (size_t)st * F::A_BYTES) +
                                (valid ? woff[n] : 0);
-                const uint32_t lrow =
-                    tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(ab * 256);
+                const uint32_t lrow = tmem + ((uint32_t)(quarter * 32) << 16) +
+                                      (uint32_t)(ab * 256 + mt * 128);
 #pragma unroll 1
                 for (int li = hf; li < F::LOADS; li += 2) {
                     uint32_t r[32];
@@ -526,6 +538,7 @@ __global__ void __launch_bounds__(kToepThreads, 1)
                         }
                     }
                 }
+              }
             }
             tc_fence_before();
             fence_proxy_async_smem();
@@ -569,9 +582,9 @@ template <int WS>
 bool toep_layout(const Geom& g, ToepLayout& L)
 {
     using F = ToepCfg<WS>;
-    if (g.nw < 1 || g.nw > kToepTileWindows)
+    if (g.nw < 1 || g.nw > F::TW)
         return false;
-    L.bpt = kToepTileWindows / g.nw;
+    L.bpt = F::TW / g.nw;
     L.sb = (L.bpt + 1) / 2;
     L.sub_bytes = align_up((uint32_t)L.sb * WS * g.W * 2, 128);
     uint32_t off = 0;
@@ -580,7 +593,7 @@ bool toep_layout(const Geom& g, ToepLayout& L)
     L.off_q = align_up(off, 128);
     off = L.off_q + 2 * F::Q_BYTES;
     L.off_woff = align_up(off, 16);
-    off = L.off_woff + kToepTileWindows * 4;
+    off = L.off_woff + F::TW * 4;
     L.off_tst = align_up(off, 16);
     off = L.off_tst + (uint32_t)F::TSZ * 2;
     L.off_bar = align_up(off, 16);
