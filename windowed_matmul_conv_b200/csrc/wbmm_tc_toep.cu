@@ -1,6 +1,6 @@
 // Tensor-core (tcgen05) WBMM forward and input-gradient kernel, window-major.
 //
-// The windows of a tile (128, or 256 as two M tiles when a window has at most
+// The windows of a tile (128, or 512 as four M tiles when a window has at most
 // 64 padded positions) are the GEMM's M dimension and the output positions of
 // a window its N dimension:
 //
@@ -55,9 +55,10 @@ struct ToepCfg {
     static constexpr int NP = (WS * RP + 15) / 16 * 16;      // MMA N (output columns)
     static constexpr int QROWS = (WS - 1) * RP + NP;
     static constexpr int TSZ = (2 * WS - 1) * (2 * WS - 1);
-    // 128-window M tiles per tile: two when a window is small (N <= 64), so
-    // that the per-tile fixed costs cover twice the data
-    static constexpr int MTW = NP <= 64 ? 2 : 1;
+    // 128-window M tiles per tile: four when a window is small (N <= 64), so
+    // that the per-tile fixed costs cover four times the data
+    static constexpr int MTW = NP <= 64 ? 4 : 1;
+    static constexpr int DSTEP = NP <= 64 ? 64 : 128;        // TMEM columns between M tiles
     static constexpr int TW = 128 * MTW;                     // windows per tile
     static constexpr uint32_t A_BYTES = (uint32_t)TW * KP * 2;   // one operand stage
     static constexpr uint32_t SBO_A = (uint32_t)KP * 16;     // bytes per 8-window group
@@ -394,7 +395,7 @@ __global__ void __launch_bounds__(kToepThreads, 1)
                     const uint64_t adesc0 = smem_desc(
                         smem_u32(a_base + (size_t)st * F::A_BYTES) + (uint32_t)(mt * 16) * F::SBO_A,
                         128, F::SBO_A);
-                    const uint32_t d = tmem + (uint32_t)(ab * 256 + mt * 128);
+                    const uint32_t d = tmem + (uint32_t)(ab * 256 + mt * F::DSTEP);
 #pragma unroll
                     for (int k = 0; k < F::KSTEPS; ++k)
                         mma_ss(d, adesc0 + (uint64_t)(k * 16),
@@ -511,7 +512,7 @@ __global__ void __launch_bounds__(kToepThreads, 1)
                 uint16_t* o0 = reinterpret_cast<uint16_t*>(a_base + (size_t)st * F::A_BYTES) +
                                (valid ? woff[n] : 0);
                 const uint32_t lrow = tmem + ((uint32_t)(quarter * 32) << 16) +
-                                      (uint32_t)(ab * 256 + mt * 128);
+                                      (uint32_t)(ab * 256 + mt * F::DSTEP);
 #pragma unroll 1
                 for (int li = hf; li < F::LOADS; li += 2) {
                     uint32_t r[32];
