@@ -62,10 +62,11 @@ class Oracle:
         lib.oracle_backward_dx.argtypes = [dp, dp, dp, i, i, i, i, i]
         lib.oracle_backward_dt.argtypes = [dp, dp, dp, i, i, i, i, i]
         lib.oracle_expand.argtypes = [dp, dp, i, i]
+        lib.oracle_reparam_merge.argtypes = [dp, dp, dp, i, i, i]
         lib.oracle_dw3x3.argtypes = [dp, dp, dp, i, i, i, i]
         lib.oracle_num_threads.restype = ctypes.c_int
         for f in (lib.oracle_forward, lib.oracle_backward_dx, lib.oracle_backward_dt,
-                  lib.oracle_expand, lib.oracle_dw3x3):
+                  lib.oracle_expand, lib.oracle_reparam_merge, lib.oracle_dw3x3):
             f.restype = None
         self.lib = lib
 
@@ -107,6 +108,16 @@ class Oracle:
             raise ValueError("T must be [C, (2w-1)^2]")
         M = np.empty((C, w * w, w * w), dtype=np.float64)
         self.lib.oracle_expand(_ptr(T), _ptr(M), C, w)
+        return M
+
+    def reparam_merge(self, Tw, Tk, w, k):
+        """Inference matrix of a w-window branch plus a k-window branch (k | w)."""
+        Tw, Tk = _f64(Tw), _f64(Tk)
+        C = Tw.shape[0]
+        if w % k != 0 or Tw.shape != (C, table_size(w)) or Tk.shape != (C, table_size(k)):
+            raise ValueError("need k | w, Tw [C, (2w-1)^2] and Tk [C, (2k-1)^2]")
+        M = np.empty((C, w * w, w * w), dtype=np.float64)
+        self.lib.oracle_reparam_merge(_ptr(Tw), _ptr(Tk), _ptr(M), C, w, k)
         return M
 
     def dw3x3(self, y, K):
@@ -170,6 +181,10 @@ def backward_dt(x, dy, w):
 
 def expand(T, w):
     return default().expand(T, w)
+
+
+def reparam_merge(Tw, Tk, w, k):
+    return default().reparam_merge(Tw, Tk, w, k)
 
 
 def dw3x3(y, K):

@@ -146,6 +146,32 @@ void oracle_expand(const double *T, double *M, int C, int w)
 }
 
 /*
+ * Hierarchical window reparameterisation folded for inference (reading
+ * notes, "Method", fourth point: a k x k local structure overlaid on the
+ * w x w window, with no inference cost).  Read as a second WBMM branch of
+ * window k (k divides w) on the same input, whose windows tile each w-window
+ * 2-D; the sum of the branches is one w-window map with matrix
+ *   M[c][(p,q),(r,s)] = T_w[c, idx_w(p-r, q-s)]
+ *                       + [p/k == r/k and q/k == s/k] T_k[c, idx_k(p%k - r%k, q%k - s%k)].
+ */
+void oracle_reparam_merge(const double *Tw, const double *Tk, double *M, int C, int w, int k)
+{
+    const long tw = (long)(2 * w - 1) * (2 * w - 1), tk = (long)(2 * k - 1) * (2 * k - 1);
+    const long d = (long)w * w;
+    for (int c = 0; c < C; ++c)
+        for (int p = 0; p < w; ++p)
+            for (int q = 0; q < w; ++q)
+                for (int r = 0; r < w; ++r)
+                    for (int s = 0; s < w; ++s) {
+                        double v = Tw[(long)c * tw + rel_index(w, p - r, q - s)];
+                        if (p / k == r / k && q / k == s / k)
+                            v += Tk[(long)c * tk + rel_index(k, p % k - r % k, q % k - s % k)];
+                        M[(long)c * d * d + (long)(p * w + q) * d + (r * w + s)] = v;
+                    }
+}
+
+/*
+ * Inter-block 3x3 depthwise mixing (reading notes, "Method", third point):/*
  * Inter-block 3x3 depthwise mixing (reading notes, "Method", third point):
  * z[b,c,h,x] = sum_{a,e in 0..2} K[c,a,e] * y[b,c,h+a-1,x+e-1], with y taken
  * as zero outside the image (cross-correlation, zero padding 1, no bias).

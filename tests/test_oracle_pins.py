@@ -247,7 +247,26 @@ def pin_dw3x3(orc):
     np.testing.assert_allclose(orc.dw3x3(x, K), ref, rtol=1e-12, atol=1e-12)
 
 
-OTHER_PINS = [pin_expand, pin_dw3x3]
+def pin_reparam_merge(orc):
+    # no small branch: the expansion of the big table (pinned above)
+    Tw = rnd((2, 49), 97)
+    assert np.array_equal(orc.reparam_merge(Tw, np.zeros((2, 9)), 4, 2), orc.expand(Tw, 4))
+    # equal windows: the tables simply add
+    Tk = rnd((2, 49), 98)
+    np.testing.assert_allclose(orc.reparam_merge(Tw, Tk, 4, 4), orc.expand(Tw + Tk, 4),
+                               rtol=1e-15, atol=1e-15)
+    # the folded matrix computes the sum of the two branches: a w-window WBMM
+    # and a k-window WBMM on the same map
+    for w, k in ((4, 2), (6, 3), (6, 2), (14, 7)):
+        x = rnd((2, 3, 2 * w, w), 100 + w + k)
+        Tw = rnd((3, (2 * w - 1) ** 2), 101 + w)
+        Tk = rnd((3, (2 * k - 1) ** 2), 102 + k)
+        np.testing.assert_allclose(Oracle.forward_cached(x, orc.reparam_merge(Tw, Tk, w, k), w),
+                                   orc.forward(x, Tw, w) + orc.forward(x, Tk, k),
+                                   rtol=1e-12, atol=1e-12)
+
+
+OTHER_PINS = [pin_expand, pin_dw3x3, pin_reparam_merge]
 ALL_PINS = FORWARD_PINS + GRADIENT_PINS + OTHER_PINS
 
 
@@ -325,6 +344,14 @@ MUTANTS = [
      "for (int r = 1; r < w; ++r)", GRADIENT_PINS),
     ("dw_flipped_kernel", "oracle_dw3x3", "Kc[a * 3 + e]", "Kc[e * 3 + a]", OTHER_PINS),
     ("dw_shifted_row", "oracle_dw3x3", "const int hh = h + a - 1", "const int hh = h + a - 2",
+     OTHER_PINS),
+    ("rp_row_blocks_only", "oracle_reparam_merge", "p / k == r / k && q / k == s / k",
+     "p / k == r / k", OTHER_PINS),
+    ("rp_transposed_small", "oracle_reparam_merge",
+     "rel_index(k, p % k - r % k, q % k - s % k)", "rel_index(k, q % k - s % k, p % k - r % k)",
+     OTHER_PINS),
+    ("rp_flipped_small", "oracle_reparam_merge",
+     "rel_index(k, p % k - r % k, q % k - s % k)", "rel_index(k, r % k - p % k, s % k - q % k)",
      OTHER_PINS),
 ]
 
