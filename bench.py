@@ -43,6 +43,7 @@ WORKLOADS = {
     "sweep14": "sweep_w14",
     "sweep28": "sweep_w28",
     "cached": "hires_cached_dw",
+    "reparam": "hires_reparam",
 }
 
 
@@ -87,6 +88,8 @@ def step_bytes(wl):
         return 5 * m + tbl + wl.C * wl.t * 4          # x, y, dY, x, dX, T, dT
     if wl.kind == "cached_dw":
         return 2 * m + wl.C * wl.d * wl.d * e + wl.C * 9 * e   # x, z, M, K
+    if wl.kind == "reparam":
+        return 2 * m + wl.C * wl.d * wl.d * e                  # x, y, merged M
     return 2 * m + tbl
 
 
@@ -98,6 +101,7 @@ def kernel_bytes(wl, name):
             "backward_dt": 2 * m + wl.C * wl.t * 4,
             "forward_cached": 2 * m + wl.C * wl.d * wl.d * e,
             "forward_cached_dw3x3": 2 * m + wl.C * wl.d * wl.d * e + wl.C * 9 * e,
+            "reparam_merge": wl.C * wl.d * wl.d * e + tbl,
             "dw3x3": 2 * m + wl.C * 9 * e}[name]
 
 
@@ -107,6 +111,8 @@ def kernel_flops(wl, name):
         return 18.0 * n
     if name == "forward_cached_dw3x3":
         return 2.0 * n * wl.d + 18.0 * n
+    if name == "reparam_merge":
+        return float(wl.C * wl.d * wl.d)
     return 2.0 * n * wl.d
 
 
@@ -194,6 +200,10 @@ class Arm:
             self.dT = torch.empty((wl.C, wl.t), dtype=torch.float32, device=dev)
             nbytes = wb.wbmm_backward_workspace_bytes(wl.B, wl.C, wl.H, wl.W, wl.w, torch.bfloat16)
             self.ws = torch.empty(max(1, nbytes // 4), dtype=torch.float32, device=dev)
+        if wl.kind == "reparam":
+            self.Tk = d["Tk"].to(dev)
+            self.M = wb.reparam_merge(self.T, self.Tk, wl.w, synth.REPARAM_SMALL_WINDOW)
+            self.M2 = torch.empty_like(self.M)     # target of the timed merges
         if wl.kind == "cached_dw":
             self.M = wb.cache_matrices(self.T, wl.w)
             self.K = d["K"].to(dev)
@@ -207,12 +217,16 @@ class Arm:
             return ["forward", "backward_dx", "backward_dt"]
         if k == "cached_dw":
             return ["forward_cached", "dw3x3"]
+        if k == "reparam":
+            return ["forward_cached"]
         return ["forward"]
 
     def alternatives(self):
         """Other launches of the same step, timed for reference only: the
         fused cached forward + 3x3 (one launch; slower on 224x224 planes,
         where its stencil work blocks the epilogue warps)."""
+        if self.wl.kind == "reparam":
+            return ["reparam_merge"]    # one-time preparation of the inference matrix
         return ["forward_cached_dw3x3"] if self.wl.kind == "cached_dw" else []
 
     def calls(self):
@@ -236,6 +250,8 @@ class Arm:
             wb.wbmm_forward_cached(s["x"], self.M, None, s["y"], w)
         elif name == "forward_cached_dw3x3":
             wb.wbmm_forward_cached(s["x"], self.M, self.K, s["z"], w)
+        elif name == "reparam_merge":
+            wb.wbmm_reparam_merge(self.T, self.Tk, self.M2, w, synth.REPARAM_SMALL_WINDOW)
         elif name == "dw3x3":
             wb.wbmm_dw3x3(s["y"], self.K, s["z"])
 
@@ -306,6 +322,9 @@ def cpu_baseline(wl, host, budget_s=10.0):
             M = oracle.expand(T, wl.w)
             y = oracle.forward_cached(x, M, wl.w)
             oracle.dw3x3(y, host["K"])
+        elif wl.kind == "reparam":
+            M = oracle.reparam_merge(T, host["Tk"], wl.w, synth.REPARAM_SMALL_WINDOW)
+            oracle.forward_cached(x, M, wl.w)
         else:
             oracle.forward(x, T, wl.w)
         runs += 1
@@ -414,7 +433,8 @@ def run_gpu(args, rank, world, local_rank):
     if wl.kind == "train":
         host_in["dY"] = wb_arm.host["dY"].pin_memory()
     s0 = wb_arm.sets[0]
-    outs = ["y"] if wl.kind == "forward" else (["y", "dX"] if wl.kind == "train" else ["z"])
+    outs = (["y"] if wl.kind in ("forward", "reparam")
+            else (["y", "dX"] if wl.kind == "train" else ["z"]))
     host_out = {o: torch.empty(s0[o].shape, dtype=s0[o].dtype, pin_memory=True) for o in outs}
     if wl.kind == "train":
         host_out["dT"] = torch.empty(wb_arm.dT.shape, dtype=torch.float32, pin_memory=True)
@@ -457,7 +477,8 @@ def run_gpu(args, rank, world, local_rank):
             "workload": "%s: B%d C%d %dx%d w%d (%s)" % (wl.name, wl.B, wl.C, wl.H, wl.W, wl.w,
                                                       {"train": "forward + dX + dT",
                                                        "forward": "forward",
-                                                       "cached_dw": "cached forward, then 3x3"}[wl.kind]),
+                                                       "cached_dw": "cached forward, then 3x3",
+                                                       "reparam": "cached forward with the merged 14x14 + 7x7 matrix"}[wl.kind]),
             "B": wl.B, "C_per_gpu": wl.C, "H": wl.H, "W": wl.W, "w": wl.w,
             "parallelism": "channel-sharded, %d rank(s), no collective" % world,
             "channels_of_rank0": list(channel_range(wl.C * world, world, 0)),
@@ -530,6 +551,9 @@ def run_reference(args, rank, world):
         elif wl.kind == "cached_dw":
             y = oracle.forward_cached(x, oracle.expand(T, wl.w), wl.w)
             oracle.dw3x3(y, d["K"])
+        elif wl.kind == "reparam":
+            M = oracle.reparam_merge(T, d["Tk"], wl.w, synth.REPARAM_SMALL_WINDOW)
+            oracle.forward_cached(x, M, wl.w)
         else:
             oracle.forward(x, T, wl.w)
 

@@ -115,6 +115,23 @@ WBMM_API wbmm_status wbmm_cache_matrices(const void *T, void *M, int C, int w,
                                 wbmm_dtype dt, void *stream);
 
 /*
+ * Hierarchical window reparameterisation folded for inference (reading
+ * notes, "Method", fourth point: a k x k local structure overlaid on the
+ * w x w window at no inference cost).  Read as a second WBMM branch of window
+ * k (k divides w) on the same input, whose k-windows tile every w-window; the
+ * two branches sum to one w-window map whose per-channel matrix is
+ *   M[c][(p,q),(r,s)] = Tw[c, (p-r+w-1)(2w-1) + (q-s+w-1)]
+ *     + (p/k == r/k and q/k == s/k) * Tk[c, (p%k-r%k+k-1)(2k-1) + (q%k-s%k+k-1)]
+ * (rows and columns u = p*w+q), summed in fp32 and rounded once to dt.  Pass
+ * M to wbmm_forward_cached.
+ *   Tw [C,(2w-1)^2], Tk [C,(2k-1)^2], M [C,w*w,w*w]; dtype dt.
+ * Errors: INVALID_ARG (null pointer, C, w or k <= 0, k not dividing w, M
+ * overlapping a table), UNSUPPORTED (w > 64), DTYPE, ALIGNMENT, CUDA.
+ */
+WBMM_API wbmm_status wbmm_reparam_merge(const void *Tw, const void *Tk, void *M, int C, int w,
+                                        int k, wbmm_dtype dt, void *stream);
+
+/*
  * Cached-matrix forward, optionally followed by the inter-block 3x3 depthwise
  * mixing (reading notes, "Method", third point):
  *   y = M_c X_c per window (M as written by wbmm_cache_matrices, or any

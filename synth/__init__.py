@@ -62,7 +62,12 @@ WORKLOADS = {
     "sweep_w28": Workload("sweep_w28", 32, 256, 112, 112, 28, "bf16", "normal", "forward"),
     "hires_cached_dw": Workload("hires_cached_dw", 8, 96, 224, 224, 14, "bf16", "normal",
                                 "cached_dw"),
+    # inference with a 14x14 and a 7x7 branch folded into one matrix
+    "hires_reparam": Workload("hires_reparam", 8, 96, 224, 224, 14, "bf16", "normal", "reparam"),
 }
+
+# second branch window of the "reparam" workloads
+REPARAM_SMALL_WINDOW = 7
 
 
 def torch_dtype(name):
@@ -98,6 +103,10 @@ def draw(wl: Workload, seed: int = 0):
     if wl.kind == "cached_dw":
         out["K"] = (torch.randn((wl.C, 1, 3, 3), generator=gen, dtype=torch.float32)
                     * DW_SIGMA).to(dt)
+    if wl.kind == "reparam":
+        k = REPARAM_SMALL_WINDOW
+        out["Tk"] = (torch.randn((wl.C, (2 * k - 1) ** 2), generator=gen, dtype=torch.float32)
+                     * TABLE_SIGMA).to(dt)
     return out
 
 

@@ -150,6 +150,49 @@ def test_forward_cached_bf16(shape):
     check_bf16(to_np(y2), ref, bound, "cached random M")
 
 
+@pytest.mark.parametrize("dtype,w,k", [(torch.bfloat16, 14, 7), (torch.float32, 14, 7),
+                                       (torch.bfloat16, 12, 4), (torch.float32, 6, 3)])
+def test_reparam_merge(dtype, w, k):
+    C = 3
+    Tw = gen((C, (2 * w - 1) ** 2), 30, dtype, 0.02)
+    Tk = gen((C, (2 * k - 1) ** 2), 31, dtype, 0.02)
+    M = wb.reparam_merge(Tw, Tk, w, k)
+    torch.cuda.synchronize()
+    ref = oracle.reparam_merge(to_np(Tw), to_np(Tk), w, k)
+    # the sum of two stored values is exact in fp32 here, so both sides round
+    # it once to the storage type
+    exp = torch.from_numpy(ref).to(torch.float32).to(dtype).to(DEV)
+    assert torch.equal(M, exp)
+    # the merged matrix computes the two branches: w-window plus k-window WBMM
+    x = gen((2, C, 2 * w, 2 * w), 32, dtype)
+    y = wb.forward_cached(x, M, w)
+    torch.cuda.synchronize()
+    xr = to_np(x)
+    ref_y = oracle.forward(xr, to_np(Tw), w) + oracle.forward(xr, to_np(Tk), k)
+    Mn = to_np(M)
+    rn = np.sqrt((Mn ** 2).sum(axis=2)).reshape(C, w, w)
+    bound = window_norms(xr, w) * np.tile(rn, (1, 2, 2))[None]
+    if dtype == torch.bfloat16:
+        check_bf16(to_np(y), ref_y, bound, "reparam forward")
+    else:
+        absref = oracle.forward_cached(np.abs(xr), np.abs(Mn), w)
+        check_f32(to_np(y), ref_y, absref, "reparam forward")
+
+
+def test_reparam_merge_argument_errors():
+    Tw = gen((2, 27 * 27), 33, scale=0.02)
+    Tk = gen((2, 9 * 9), 34, scale=0.02)
+    M = torch.empty((2, 196, 196), dtype=torch.bfloat16, device=DEV)
+    before = wb.wbmm_launch_count()
+    with pytest.raises(wb.WbmmError) as e:
+        wb.wbmm_reparam_merge(Tw, Tk, M, 14, 5)       # 5 does not divide 14
+    assert e.value.status == 1
+    with pytest.raises(wb.WbmmError) as e:
+        wb.wbmm_reparam_merge(Tw, Tk, Tw, 14, 7)      # output overlaps a table
+    assert e.value.status == 1
+    assert wb.wbmm_launch_count() == before
+
+
 # (B, C, H, W, w): fused work units of one tile holding several planes
 # (56x56, 48x48 at w=16) and of one plane spanning several tiles (112x56 at
 # w=7, 224x224)

@@ -10,8 +10,8 @@ runs in the library's CUDA kernels.  Importing this package fails loudly if
 the library has not been built (``python windowed_matmul_conv_b200/build.py``).
 
 The convenience functions ``forward``, ``backward``, ``cache_matrices``,
-``forward_cached`` and ``dw3x3`` allocate outputs with torch and call the
-entry points above.
+``reparam_merge``, ``forward_cached`` and ``dw3x3`` allocate outputs with
+torch and call the entry points above.
 """
 import ctypes
 import os
@@ -33,7 +33,7 @@ STATUS_NAMES = {0: "WBMM_OK", 1: "WBMM_ERR_INVALID_ARG", 2: "WBMM_ERR_SHAPE",
                 3: "WBMM_ERR_DTYPE", 4: "WBMM_ERR_ALIGNMENT", 5: "WBMM_ERR_UNSUPPORTED",
                 6: "WBMM_ERR_WORKSPACE", 7: "WBMM_ERR_CUDA", 8: "WBMM_ERR_TIMEOUT"}
 EXPORTS = ("wbmm_forward", "wbmm_backward_workspace_bytes", "wbmm_backward",
-           "wbmm_cache_matrices", "wbmm_forward_cached", "wbmm_dw3x3",
+           "wbmm_cache_matrices", "wbmm_reparam_merge", "wbmm_forward_cached", "wbmm_dw3x3",
            "wbmm_get_device_status", "wbmm_status_string", "wbmm_set_wait_budget",
            "wbmm_wait_selftest", "wbmm_launch_count", "wbmm_last_path",
            "wbmm_backward_dt_static")
@@ -44,6 +44,7 @@ _lib.wbmm_backward_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, _i]
 _lib.wbmm_backward_workspace_bytes.restype = _sz
 _lib.wbmm_backward.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _sz, _i, _i, _i, _i, _i, _i, _vp]
 _lib.wbmm_cache_matrices.argtypes = [_vp, _vp, _i, _i, _i, _vp]
+_lib.wbmm_reparam_merge.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _vp]
 _lib.wbmm_backward_dt_static.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]
 _lib.wbmm_forward_cached.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]
 _lib.wbmm_dw3x3.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]
@@ -57,8 +58,7 @@ _lib.wbmm_launch_count.argtypes = []
 _lib.wbmm_launch_count.restype = ctypes.c_ulonglong
 _lib.wbmm_last_path.argtypes = []
 for _f in ("wbmm_forward", "wbmm_backward", "wbmm_backward_dt_static", "wbmm_cache_matrices",
-           "wbmm_forward_cached",
-           "wbmm_dw3x3", "wbmm_get_device_status", "wbmm_wait_selftest", "wbmm_last_path"):
+           "wbmm_reparam_merge", "wbmm_forward_cached", "wbmm_dw3x3", "wbmm_get_device_status", "wbmm_wait_selftest", "wbmm_last_path"):
     getattr(_lib, _f).restype = _i
 
 
@@ -185,6 +185,19 @@ def backward(x, T, dY, w, need_dx=True, need_dt=True, stream=None):
         ws = torch.empty(max(1, nbytes // 4), dtype=torch.float32, device=dY.device)
     wbmm_backward(x, T, dY, dX, dT, ws, w, stream)
     return dX, dT
+
+
+def wbmm_reparam_merge(Tw, Tk, M, w, k, stream=None):
+    _check(_lib.wbmm_reparam_merge(_p(Tw), _p(Tk), _p(M), int(Tw.shape[0]), int(w), int(k),
+                                   _dt(Tw), _stream(stream)))
+
+
+def reparam_merge(Tw, Tk, w, k, stream=None):
+    """Inference matrix [C, w*w, w*w] of a w-window branch (table Tw) plus a
+    k-window branch (table Tk), k dividing w; feed it to forward_cached."""
+    M = torch.empty((Tw.shape[0], w * w, w * w), dtype=Tw.dtype, device=Tw.device)
+    wbmm_reparam_merge(Tw, Tk, M, w, k, stream)
+    return M
 
 
 def cache_matrices(T, w, stream=None):

@@ -303,6 +303,30 @@ wbmm_status wbmm_cache_matrices(const void* T, void* M, int C, int w, wbmm_dtype
     return from_cuda(cache_matrices_launch(C, w, dt == WBMM_BF16, T, M, L));
 }
 
+wbmm_status wbmm_reparam_merge(const void* Tw, const void* Tk, void* M, int C, int w, int k,
+                               wbmm_dtype dt, void* stream)
+{
+    if (!dtype_ok(dt))
+        return WBMM_ERR_DTYPE;
+    if (!Tw || !Tk || !M || C <= 0 || w <= 0 || k <= 0 || w % k != 0)
+        return WBMM_ERR_INVALID_ARG;
+    if (w > 64)
+        return WBMM_ERR_UNSUPPORTED;
+    if (!aligned(Tw, dt) || !aligned(Tk, dt) || !aligned(M, dt))
+        return WBMM_ERR_ALIGNMENT;
+    const size_t d = (size_t)w * w;
+    const size_t tw = (size_t)(2 * w - 1) * (2 * w - 1), tk = (size_t)(2 * k - 1) * (2 * k - 1);
+    const Span ms{M, (size_t)C * d * d * elem_size(dt)};
+    if (overlap(ms, Span{Tw, C * tw * elem_size(dt)}) ||
+        overlap(ms, Span{Tk, C * tk * elem_size(dt)}))
+        return WBMM_ERR_INVALID_ARG;
+    Launch L;
+    wbmm_status st = make_launch(stream, &L);
+    if (st != WBMM_OK)
+        return st;
+    return from_cuda(reparam_merge_launch(C, w, k, dt == WBMM_BF16, Tw, Tk, M, L));
+}
+
 wbmm_status wbmm_forward_cached(const void* x, const void* M, const void* dw3x3, void* out,
                                 int B, int C, int H, int W, int w, wbmm_dtype dt, void* stream)
 {

@@ -86,6 +86,8 @@ cudaError_t dt_finalize_launch(int C, int tsz, int chunks, const float* partials
                                const Launch& L);
 cudaError_t cache_matrices_launch(int C, int w, bool is_bf16, const void* T, void* M,
                                   const Launch& L);
+cudaError_t reparam_merge_launch(int C, int w, int k, bool is_bf16, const void* Tw,
+                                 const void* Tk, void* M, const Launch& L);
 cudaError_t dw3x3_launch(const Geom& g, bool is_bf16, const void* y, const void* K, void* z,
                          const Launch& L);
 cudaError_t wait_selftest_launch(unsigned long long cycles, const Launch& L);

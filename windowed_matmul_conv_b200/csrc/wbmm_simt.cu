@@ -156,6 +156,31 @@ __global__ void __launch_bounds__(256) simt_fwd_rows_kernel(const TIn* __restric
     }
 }
 
+// ------------------------------------------- reparameterisation merge
+// One thread per matrix entry: the w-window table entry plus, inside the
+// same k x k sub-window, the k-window table entry; fp32 sum, one rounding.
+template <typename E>
+__global__ void reparam_kernel(const E* __restrict__ Tw, const E* __restrict__ Tk,
+                               E* __restrict__ M, int C, int w, int k)
+{
+    grid_dep_wait();
+    grid_dep_launch();
+    const int d = w * w, Lw = 2 * w - 1, Lk = 2 * k - 1;
+    const long long total = (long long)C * d * d;
+    for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < total;
+         e += (long long)gridDim.x * blockDim.x) {
+        const int c = (int)(e / ((long long)d * d));
+        const int rem = (int)(e - (long long)c * d * d);
+        const int u = rem / d, v = rem - (rem / d) * d;
+        const int p = u / w, q = u - (u / w) * w, r = v / w, s = v - (v / w) * w;
+        float val = to_f(Tw[(long long)c * Lw * Lw + (p - r + w - 1) * Lw + (q - s + w - 1)]);
+        if (p / k == r / k && q / k == s / k)
+            val += to_f(Tk[(long long)c * Lk * Lk + (p % k - r % k + k - 1) * Lk +
+                           (q % k - s % k + k - 1)]);
+        M[e] = from_f<E>(val);
+    }
+}
+
 // ------------------------------------------------------- table gradient
 // One block per (channel, chunk of kSimtChunkBands bands); each thread owns
 // table bins and sums dy[p,q] * x[p-dp, q-dq] over the chunk's windows in a
@@ -534,6 +559,32 @@ cudaError_t cache_matrices_launch(int C, int w, bool is_bf16, const void* T, voi
     else
         e = launch_pdl(cache_kernel<uint32_t>, grid, block, 0, L.stream,
                        static_cast<const uint32_t*>(T), static_cast<uint32_t*>(M), C, w);
+    if (e != cudaSuccess)
+        return e;
+    note_launches(1);
+    return cudaGetLastError();
+}
+
+cudaError_t reparam_merge_launch(int C, int w, int k, bool is_bf16, const void* Tw,
+                                 const void* Tk, void* M, const Launch& L)
+{
+    const long long total = (long long)C * w * w * w * w;
+    long long blocks = (total + 255) / 256;
+    if (blocks > (long long)L.num_sms * 32)
+        blocks = (long long)L.num_sms * 32;
+    if (blocks < 1)
+        return cudaSuccess;
+    const dim3 grid((unsigned)blocks), block(256);
+    cudaError_t e;
+    if (is_bf16) {
+        using E = __nv_bfloat16;
+        e = launch_pdl(reparam_kernel<E>, grid, block, 0, L.stream, static_cast<const E*>(Tw),
+                       static_cast<const E*>(Tk), static_cast<E*>(M), C, w, k);
+    } else {
+        e = launch_pdl(reparam_kernel<float>, grid, block, 0, L.stream,
+                       static_cast<const float*>(Tw), static_cast<const float*>(Tk),
+                       static_cast<float*>(M), C, w, k);
+    }
     if (e != cudaSuccess)
         return e;
     note_launches(1);
