@@ -117,6 +117,71 @@ def test_dt_is_deterministic():
         assert torch.equal(r, runs[0])
 
 
+# Degenerate and boundary window sizes: w = 1 (each channel a scalar gain,
+# CUDA-core path), one window per image (tensor-core path, nh = nw = 1),
+# w = 32 (largest register-tiled CUDA-core size) and w = 40 (plain CUDA-core
+# kernel), forward and both gradients against the oracle.
+EDGE_SHAPES = [(2, 3, 5, 7, 1, torch.bfloat16), (2, 3, 5, 7, 1, torch.float32),
+               (3, 2, 14, 14, 14, torch.bfloat16), (1, 2, 64, 32, 32, torch.bfloat16),
+               (1, 2, 40, 40, 40, torch.float32)]
+
+
+@pytest.mark.parametrize("shape", EDGE_SHAPES, ids=lambda s: "x".join(map(str, s[:5])) + str(s[5])[-4:])
+def test_edge_window_sizes(shape):
+    B, C, H, W, w, dtype = shape
+    x = gen((B, C, H, W), 40, dtype)
+    dy = gen((B, C, H, W), 41, dtype)
+    T = gen((C, (2 * w - 1) ** 2), 42, dtype, 0.02)
+    y = run_forward(x, T, w)
+    dX, dT = wb.backward(x, T, dy, w)
+    torch.cuda.synchronize()
+    assert wb.wbmm_get_device_status() == 0
+    xr, gr, Tr = to_np(x), to_np(dy), to_np(T)
+    if dtype == torch.bfloat16:
+        check_bf16(to_np(y), oracle.forward(xr, Tr, w), forward_rowbound(xr, Tr, w), "y")
+        check_bf16(to_np(dX), oracle.backward_dx(gr, Tr, w),
+                   forward_rowbound(gr, Tr[:, ::-1].copy(), w), "dX")
+        check_bf16(to_np(dT), oracle.backward_dt(xr, gr, w), dt_bound(xr, gr, w), "dT")
+    else:
+        check_f32(to_np(y), oracle.forward(xr, Tr, w),
+                  oracle.forward(np.abs(xr), np.abs(Tr), w), "y")
+        check_f32(to_np(dX), oracle.backward_dx(gr, Tr, w),
+                  oracle.backward_dx(np.abs(gr), np.abs(Tr), w), "dX")
+        check_f32(to_np(dT), oracle.backward_dt(xr, gr, w),
+                  oracle.backward_dt(np.abs(xr), np.abs(gr), w), "dT")
+    if w == 1:
+        # one-position windows: y = T_c * x exactly (one product, rounded once)
+        exp = (x.float() * T.float()[:, 0].view(1, C, 1, 1)).to(dtype)
+        assert torch.equal(y, exp)
+
+
+def test_unsupported_and_empty_shapes_launch_nothing():
+    x = gen((1, 1, 65, 65), 43)
+    T = gen((1, 129 * 129), 44, scale=0.02)
+    y = torch.empty_like(x)
+    before = wb.wbmm_launch_count()
+    with pytest.raises(wb.WbmmError) as e:
+        wb.wbmm_forward(x, T, y, 65)                   # w above the supported maximum
+    assert e.value.status == 5
+    with pytest.raises(wb.WbmmError) as e:             # an empty batch is rejected
+        wb._check(wb._lib.wbmm_forward(wb._p(x), wb._p(T), wb._p(y), 0, 1, 65, 65, 65, 1,
+                                       wb._stream(None)))
+    assert e.value.status == 1
+    assert wb.wbmm_launch_count() == before
+
+
+def test_full_size_fp32_forward_sampled():
+    wl = synth.WORKLOADS["fwd_f32"]
+    d = synth.draw(wl, seed=0)
+    x, T = d["x"].to(DEV), d["T"].to(DEV)
+    y = run_forward(x, T, wl.w)
+    assert wb.wbmm_last_path() == 2
+    bs, cs = sample_planes(wl.B, wl.C)
+    xs, Ts = to_np(d["x"][bs][:, cs]), to_np(d["T"][cs])
+    check_f32(to_np(y[bs][:, cs]), oracle.forward(xs, Ts, wl.w),
+              oracle.forward(np.abs(xs), np.abs(Ts), wl.w), "fp32 forward")
+
+
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 def test_cache_matrices_bit_exact(dtype):
     for w in (3, 7, 14):

@@ -500,13 +500,16 @@ cudaError_t simt_dt_launch(const Geom& g, bool is_bf16, const void* x, const voi
                            float* partials, const Launch& L)
 {
     const size_t smem = (size_t)2 * g.w * g.W * 4;
-    if (smem > kSimtSmemMax || g.tsz > 256 * kSimtMaxBinsPerThread)
+    // each thread owns up to kSimtMaxBinsPerThread table entries: 256 threads
+    // cover w <= 32, 1024 threads every w the library accepts (<= 64)
+    const int threads = g.tsz <= 256 * kSimtMaxBinsPerThread ? 256 : 1024;
+    if (smem > kSimtSmemMax || g.tsz > threads * kSimtMaxBinsPerThread)
         return cudaErrorInvalidConfiguration;
     const int chunks = simt_dt_chunks(g);
     const long long blocks = (long long)g.C * chunks;
     if (blocks == 0)
         return cudaSuccess;
-    const dim3 grid((unsigned)blocks), block(256);
+    const dim3 grid((unsigned)blocks), block(threads);
     cudaError_t e;
     if (is_bf16) {
         using E = __nv_bfloat16;
