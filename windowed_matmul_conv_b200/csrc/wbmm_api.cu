@@ -349,6 +349,12 @@ wbmm_status wbmm_forward_cached(const void* x, const void* M, const void* dw3x3,
     if ((st = make_launch(stream, &L)) != WBMM_OK)
         return st;
     const bool fused = dw3x3 != nullptr;
+    if (dt == WBMM_BF16 && !fused && tc_cached_supported(g)) {
+        st = from_cuda(tc_cached_launch(g, x, M, out, L));
+        if (st == WBMM_OK)
+            t_last_path = 1;
+        return st;
+    }
     if (dt == WBMM_BF16 && tc_fwd_supported(g, fused)) {
         st = from_cuda(tc_fwd_launch(g, kCached, x, M, out, dw3x3, L));
         if (st == WBMM_OK)

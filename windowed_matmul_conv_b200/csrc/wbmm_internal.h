@@ -64,6 +64,12 @@ bool tc_toep_supported(const Geom& g);
 cudaError_t tc_toep_launch(const Geom& g, AMode mode, const void* x, const void* T, void* y,
                            const Launch& L);
 
+// tcgen05 forward with a cached [C][d][d] matrix, windows as the MMA's M
+// dimension (no fused 3x3).
+bool tc_cached_supported(const Geom& g);
+cudaError_t tc_cached_launch(const Geom& g, const void* x, const void* M, void* y,
+                             const Launch& L);
+
 // tcgen05 table gradient: one contiguous tile range per CTA.  The workspace
 // (tc_dt_workspace_floats floats, any prior content) holds the fp32 partial
 // tables of channels split between CTAs and one flag word per table.
