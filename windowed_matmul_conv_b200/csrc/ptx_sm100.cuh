@@ -156,6 +156,20 @@ __device__ __forceinline__ bool wait_token(const unsigned long long *p, unsigned
     return true;
 }
 
+// ------------------------------------------------------- 4-byte async copies
+// Global -> shared copy of one 32-bit word, both addresses 4-byte aligned.
+// The copies of a thread complete at cp_async_wait_all().
+__device__ __forceinline__ void cp_async_4(uint32_t smem_dst, const void *gsrc)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_dst), "l"(gsrc)
+                 : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all()
+{
+    asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
 // ------------------------------------------------------- bulk async copies
 // Global -> shared, completion signalled on `bar` as transaction bytes.
 // Both addresses 16-byte aligned, bytes a multiple of 16.

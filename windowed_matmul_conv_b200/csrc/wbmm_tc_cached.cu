@@ -46,12 +46,13 @@ struct CachedCfg {
     static constexpr int KSTEPS = (WS + G - 1) / G;
     static constexpr int KP = KSTEPS * 16;
     static constexpr int RROWS = KSTEPS * G;                 // window rows incl. zero rows
-    static constexpr int NP = (WS * RP + 15) / 16 * 16;      // MMA N
-    static constexpr uint32_t SBO_B = (uint32_t)KP * 16;     // bytes per 8-row group of B
+    static constexpr int KC = KP / 8;                        // core matrices along K
+    static constexpr int NP = (D + 15) / 16 * 16;            // MMA N: output positions, dense
+    static constexpr uint32_t LBO_B = 144;                   // core matrix stride along K
+    static constexpr uint32_t SBO_B = (uint32_t)KC * LBO_B;  // bytes per 8-row group of B
     static constexpr uint32_t B_BYTES = (uint32_t)NP / 8 * SBO_B;
     static constexpr int A_COLS = KP / 2;                    // TMEM columns per A stage
     static constexpr int LOADS = (NP + 31) / 32;
-    static constexpr int RL = 32 / RP;
     static constexpr uint32_t OUT_BYTES = (uint32_t)((128 * D * 2 + 127) / 128 * 128);
     static constexpr uint32_t IDESC = idesc_bf16(128, NP);
     static_assert(A_COLS <= 128 && NP <= 256, "TMEM plan: A stages at 0/128, D at 256");
@@ -89,7 +90,6 @@ struct CachedBars {
     uint64_t acc_empty;
     uint64_t out_full;
     uint64_t out_empty;
-    uint64_t m_full;        // a chunk of M_c copied into the staging buffer
     uint64_t fin;
     uint32_t tmem_slot;
     int abort;
@@ -115,37 +115,66 @@ __device__ __forceinline__ BandTile cached_half(const TcCachedParams& P, const B
     return s;
 }
 
-// B = M_c^T in the K-major operand layout: row n' = p*RP + q (output
-// position), K slot k = r*RP + s (input position); 8-row groups SBO_B bytes
-// apart, the core matrices of a group 128 bytes apart along K.  One thread
-// per (row, 8-slot group); padding rows and slots are zero.  `m` holds rows
-// u0 .. u1-1 of M_c (u = p*w+q, d entries each); items whose row lies
-// outside that range are skipped, so B can be built in row chunks.
+// B = M_c^T in the K-major operand layout: row n = p*w + q (output position
+// p, q; row n of M_c), K slot k = r*RP + s (input position r, s), the same K
+// order as the table path, so both give identical bits.  Core matrices
+// (8 rows x 16 bytes) lie LBO_B = 144 bytes apart along K and SBO_B apart
+// along N: the 16 spare bytes put consecutive core matrices of one row on
+// different bank groups, so copying rows of M_c in order writes shared
+// memory almost without conflicts.  The whole image is zeroed once per
+// launch (zero_b, then a barrier among the builders); a build rewrites only
+// the d x d values.
 template <int WS>
-__device__ __forceinline__ void build_b_rows(uint8_t* b, const uint16_t* m, int u0, int u1, int tid,
-                                             int nthreads)
+__device__ __forceinline__ void zero_b(uint8_t* b, int tid, int nthreads)
 {
     using F = CachedCfg<WS>;
-    constexpr int KC = F::KP / 8;
-    for (int item = tid; item < F::NP * KC; item += nthreads) {
-        const int np = item / KC, kc = item - (item / KC) * KC;
-        const int p = np / F::RP, q = np - (np / F::RP) * F::RP;
-        const int u = p * WS + q;
-        const bool row_ok = p < WS && q < WS;
-        // padding rows belong to the first chunk; real rows to theirs
-        if (row_ok ? (u < u0 || u >= u1) : (u0 != 0))
-            continue;
-        const int r = (kc * 8) / F::RP, s0 = (kc * 8) - r * F::RP;
-        uint16_t v[8];
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-            const int s = s0 + t;
-            v[t] = (row_ok && r < WS && s < WS) ? m[(long long)(u - u0) * F::D + r * WS + s]
-                                                 : (uint16_t)0;
+    for (int i = tid; i < (int)(F::B_BYTES / 16); i += nthreads)
+        reinterpret_cast<uint4*>(b)[i] = make_uint4(0u, 0u, 0u, 0u);
+}
+
+// M_c is read in its own order, so a warp's loads are coalesced.  For even
+// w a window row holds whole 32-bit pairs: one asynchronous 4-byte copy per
+// pair, all of a thread's copies in flight at once.  For odd w pairs
+// straddle window rows: 16-bit loads, eight per thread per pass, all loads
+// of a pass issued before its stores.
+template <int WS>
+__device__ __forceinline__ void build_b_global(uint8_t* b, const uint16_t* Mc, int tid,
+                                               int nthreads)
+{
+    using F = CachedCfg<WS>;
+    if constexpr (WS % 2 == 0) {
+        constexpr int HALF = F::D / 2;   // 32-bit pairs per row of M_c
+        const uint32_t b32 = smem_u32(b);
+        for (int j = tid; j < F::D * HALF; j += nthreads) {
+            const int u = j / HALF, e = 2 * (j - (j / HALF) * HALF);
+            const int k = (e / WS) * F::RP + e % WS;
+            const uint32_t dst = (uint32_t)(u >> 3) * F::SBO_B + (uint32_t)(k >> 3) * F::LBO_B +
+                                 (uint32_t)(u & 7) * 16 + (uint32_t)(k & 7) * 2;
+            cp_async_4(b32 + dst, Mc + 2 * j);
         }
-        *reinterpret_cast<uint4*>(b + (np >> 3) * F::SBO_B + kc * 128 + (np & 7) * 16) =
-            make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
-                       pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+        cp_async_wait_all();
+    } else {
+        constexpr int BATCH = 8;
+        constexpr int N = F::D * F::D;
+        for (int base = tid; base < N; base += BATCH * nthreads) {
+            uint16_t v[BATCH];
+#pragma unroll
+            for (int j = 0; j < BATCH; ++j) {
+                const int e = base + j * nthreads;
+                v[j] = e < N ? __ldg(reinterpret_cast<const unsigned short*>(Mc) + e)
+                             : (uint16_t)0;
+            }
+#pragma unroll
+            for (int j = 0; j < BATCH; ++j) {
+                const int e = base + j * nthreads;
+                if (e >= N)
+                    continue;
+                const int u = e / F::D, i = e - (e / F::D) * F::D;
+                const int k = (i / WS) * F::RP + i % WS;
+                *reinterpret_cast<uint16_t*>(b + (u >> 3) * F::SBO_B + (k >> 3) * F::LBO_B +
+                                             (u & 7) * 16 + (k & 7) * 2) = v[j];
+            }
+        }
     }
 }
 
@@ -188,7 +217,6 @@ __global__ void __launch_bounds__(kCThreads, 1)
         mbar_init(&S.acc_empty, kCEpiWarps);
         mbar_init(&S.out_full, kCEpiWarps);
         mbar_init(&S.out_empty, 1);
-        mbar_init(&S.m_full, 1);
         mbar_init(&S.fin, 1);
         S.abort = 0;
         fence_mbar_init();
@@ -280,11 +308,12 @@ __global__ void __launch_bounds__(kCThreads, 1)
                     continue;
                 tc_fence_after();
                 // K step k: A columns 8k .. 8k+7 of stage st, B core matrices 2k, 2k+1
-                const uint64_t bdesc0 = smem_desc(smem_u32(b_base), 128, F::SBO_B);
+                const uint64_t bdesc0 = smem_desc(smem_u32(b_base), F::LBO_B, F::SBO_B);
                 const uint32_t a0 = tmem + (uint32_t)(st * 128);
 #pragma unroll
                 for (int k = 0; k < F::KSTEPS; ++k)
-                    mma_ts(tmem + 256u, a0 + (uint32_t)(k * 8), bdesc0 + (uint64_t)(k * 16),
+                    mma_ts(tmem + 256u, a0 + (uint32_t)(k * 8),
+                           bdesc0 + (uint64_t)(k * 2 * F::LBO_B / 16),
                            F::IDESC, k > 0 ? 1u : 0u);
                 tc_commit(&S.a_empty[st]);
                 tc_commit(&S.acc_full);
@@ -392,40 +421,17 @@ __global__ void __launch_bounds__(kCThreads, 1)
         const int et = threadIdx.x - kCEpiWarp0 * 32;
         const int n = quarter * 32 + lane;
         const int c_first = cached_tile(P, it0).c;
-        // B of channel c.  Even w: M_c (16-byte aligned, a multiple of 16
-        // bytes) is bulk-copied into the idle staging buffer in at most two
-        // row chunks and rearranged from there; odd w reads it directly.
-        // All epilogue warps take part in every build whatever their wait
-        // results, so the named barriers always see all 256 threads.
-        int mphase = 0;
+        // B of channel c, read straight from HBM/L2.  All epilogue warps take
+        // part in every build whatever their wait results.
         auto build_for = [&](int c) {
-            const uint16_t* Mc = P.M + (long long)c * F::D * F::D;
-            if (WS % 2 == 0) {
-                constexpr int U0 = F::D * F::D * 2 <= (int)F::OUT_BYTES ? F::D : (F::D / 2 + 7) / 8 * 8;
-                for (int part = 0; part < 2; ++part) {
-                    const int u0 = part == 0 ? 0 : U0, u1 = part == 0 ? U0 : F::D;
-                    if (u0 >= u1)
-                        break;
-                    named_bar_sync(2, kCEpiWarps * 32);     // staging free
-                    if (et == 0) {
-                        const uint32_t bytes = (uint32_t)(u1 - u0) * F::D * 2;
-                        mbar_arrive_expect_tx(&S.m_full, bytes);
-                        bulk_g2s(out_base, Mc + (long long)u0 * F::D, bytes, &S.m_full);
-                    }
-                    mbar_wait(&S.m_full, mphase & 1, abort, P.budget, P.status);
-                    ++mphase;
-                    build_b_rows<WS>(b_base, reinterpret_cast<const uint16_t*>(out_base), u0, u1,
-                                     et, kCEpiWarps * 32);
-                }
-                named_bar_sync(2, kCEpiWarps * 32);         // staging read before reuse
-            } else {
-                build_b_rows<WS>(b_base, Mc, 0, F::D, et, kCEpiWarps * 32);
-            }
+            build_b_global<WS>(b_base, P.M + (long long)c * F::D * F::D, et, kCEpiWarps * 32);
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0)
                 mbar_arrive(&S.b_full);
         };
+        zero_b<WS>(b_base, et, kCEpiWarps * 32);
+        named_bar_sync(1, kCEpiWarps * 32);
         build_for(c_first);
         for (int seq = 0; seq < n_it; ++seq) {
             const BandTile t = cached_tile(P, it0 + seq);
@@ -440,29 +446,31 @@ __global__ void __launch_bounds__(kCThreads, 1)
                 const bool valid = n < nwin;
                 uint16_t* o0 = reinterpret_cast<uint16_t*>(out_base) + (valid ? woff[n] : 0);
                 const uint32_t lrow = tmem + ((uint32_t)(quarter * 32) << 16) + 256u;
-#pragma unroll 1
-                for (int li = hf; li < F::LOADS; li += 2) {
+                // accumulator column n is output position (n / w, n % w)
+#pragma unroll
+                for (int li = 0; li < F::LOADS; ++li) {
+                    if ((li & 1) != hf)
+                        continue;
                     uint32_t r[32];
                     tmem_ld32(lrow + (uint32_t)(li * 32), r);
                     tmem_wait_ld(r);
-                    if (valid) {
+                    if (!valid)
+                        continue;
+                    if (WS % 2 == 0) {
 #pragma unroll
-                        for (int rr = 0; rr < F::RL; ++rr) {
-                            const int pr = li * F::RL + rr;
-                            if (pr < WS) {
-                                uint16_t* o = o0 + pr * P.W;
-                                if (WS % 2 == 0) {
+                        for (int j = 0; j < 32; j += 2) {
+                            const int e = li * 32 + j;
+                            if (e < F::D)
+                                *reinterpret_cast<uint32_t*>(o0 + (e / WS) * P.W + e % WS) =
+                                    cbf16x2_rn(r[j], r[j + 1]);
+                        }
+                    } else {
 #pragma unroll
-                                    for (int m = 0; m < WS / 2; ++m)
-                                        reinterpret_cast<uint32_t*>(o)[m] = cbf16x2_rn(
-                                            r[rr * F::RP + 2 * m], r[rr * F::RP + 2 * m + 1]);
-                                } else {
-#pragma unroll
-                                    for (int s = 0; s < WS; ++s)
-                                        o[s] = __bfloat16_as_ushort(__float2bfloat16_rn(
-                                            __uint_as_float(r[rr * F::RP + s])));
-                                }
-                            }
+                        for (int j = 0; j < 32; ++j) {
+                            const int e = li * 32 + j;
+                            if (e < F::D)
+                                o0[(e / WS) * P.W + e % WS] =
+                                    __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(r[j])));
                         }
                     }
                 }
@@ -475,13 +483,9 @@ __global__ void __launch_bounds__(kCThreads, 1)
                 mbar_arrive(&S.out_full);
             }
             // the channel's last tile is done: every MMA that read B has
-            // completed (acc_full), so B can take the next channel's matrix;
-            // the staging buffer is free once the storer has read this tile
-            if (seq + 1 < n_it && cached_tile(P, it0 + seq + 1).c != t.c) {
-                if (WS % 2 == 0)
-                    mbar_wait(&S.out_empty, seq & 1, abort, P.budget, P.status);
+            // completed (acc_full), so B can take the next channel's matrix
+            if (seq + 1 < n_it && cached_tile(P, it0 + seq + 1).c != t.c)
                 build_for(t.c + 1);
-            }
         }
     }
 
