@@ -19,20 +19,27 @@
 // rows of 32 bytes, 13.5 KB at w = 14, so two channels' Q fit in shared
 // memory and a channel change never stalls the tensor core.
 //
-// Warp roles (608 threads):
+// The windows (the A operand) live in tensor memory: the transform warps
+// write them there with tcgen05.st (lane = window, one 32-bit column per pair
+// of K slots), so shared memory holds only Q, the raw load ring and two
+// output staging buffers, and a tile's input and output never share a buffer.
+//
+// Warp roles (480 threads):
 //   warp 0       producer: bulk/TMA copies of half tiles (whole bands) into a
 //                ring of raw slots
 //   warp 1       MMA issuer (one thread) and TMEM owner
-//   warp 2       storer: stores a finished tile from its operand stage
-//   warps 3..10  transform: raw band layout -> K-major operand rows
-//   warps 11..18 epilogue: TMEM -> bf16 output rows -> band layout, written
-//                over the tile's own operand stage (the MMA has finished
-//                reading it), from where the storer sends it to HBM.  They
-//                also write Q: the CTA's first two channels up front, and
-//                Q of channel ci+1 right after the first tile of channel
-//                ci, whose completion implies that every MMA of channel
-//                ci-1 (the other buffer's user) has finished.
+//   warp 2       storer: stores a finished tile from its output buffer
+//   warps 3..6   transform: one per TMEM lane quarter; thread = window, raw
+//                band layout -> A rows in TMEM (two A stages)
+//   warps 7..14  epilogue: TMEM -> bf16 output rows -> band layout in an
+//                output buffer.  They also write Q: the CTA's first two
+//                channels up front, and Q of channel ci+1 right after the
+//                first tile of channel ci, whose completion implies that
+//                every MMA of channel ci-1 (the other buffer's user) has
+//                finished.
 //
+// TMEM: A stages at columns 0 and 128 (M tile mt of a stage at mt*KP/2), the
+// accumulator (single; M tile mt at 256 + mt*DSTEP).
 // Every wait is bounded; a wait that runs out raises the CTA's abort flag and
 // the device status word, and every role then runs its loop without doing
 // work so that all threads reach the drain and the TMEM release.
@@ -58,22 +65,22 @@ struct ToepCfg {
     // 128-window M tiles per tile: four when a window is small (N <= 64), so
     // that the per-tile fixed costs cover four times the data
     static constexpr int MTW = NP <= 64 ? 4 : 1;
-    static constexpr int DSTEP = NP <= 64 ? 64 : 128;        // TMEM columns between M tiles
+    static constexpr int DSTEP = NP <= 64 ? 64 : 256;        // accumulator columns per M tile
     static constexpr int TW = 128 * MTW;                     // windows per tile
-    static constexpr uint32_t A_BYTES = (uint32_t)TW * KP * 2;   // one operand stage
-    static constexpr uint32_t SBO_A = (uint32_t)KP * 16;     // bytes per 8-window group
+    static constexpr int A_COLS = KP / 2;                    // TMEM columns per M tile of A
     static constexpr uint32_t Q_BYTES = (uint32_t)QROWS * 32;
+    static constexpr uint32_t OUT_BYTES = (uint32_t)((TW * D * 2 + 127) / 128 * 128);
     static constexpr int LOADS = (NP + 31) / 32;             // 32-column TMEM loads per row
     static constexpr int RL = 32 / RP;                       // window rows per load
     static constexpr uint32_t IDESC = idesc_bf16(128, NP);
-    static_assert(NP <= 256, "two accumulators of NP columns must fit in TMEM");
+    static_assert(MTW * A_COLS <= 128, "an A stage fits in 128 TMEM columns");
+    static_assert((MTW - 1) * DSTEP + NP <= 256, "the accumulator fits in 256 TMEM columns");
     static_assert((WS - 1) * RP % 8 == 0, "Q row offsets must be whole core matrices");
 };
 
 constexpr int kToepRing = 8;
-constexpr int kToepXformWarps = 8;
 constexpr int kToepXformWarp0 = 3;
-constexpr int kToepEpiWarp0 = kToepXformWarp0 + kToepXformWarps;
+constexpr int kToepEpiWarp0 = kToepXformWarp0 + 4;
 constexpr int kToepEpiWarps = 8;
 constexpr int kToepThreads = (kToepEpiWarp0 + kToepEpiWarps) * 32;
 
@@ -90,10 +97,11 @@ struct TcToepParams {
     int bands;              // bands per channel
     int items;              // C * tpc
     int R;                  // raw ring depth (half tiles)
+    int nout;               // output buffers (1 or 2)
     uint32_t sub_bytes;     // raw slot stride
     int use_tmap;
     int kimg_sub;           // planes per half tile when use_tmap
-    uint32_t off_a, off_q, off_raw, off_woff, off_bar, off_tst;
+    uint32_t off_out, off_q, off_raw, off_woff, off_bar, off_tst;
     unsigned long long budget;
     int* status;
 };
@@ -101,12 +109,13 @@ struct TcToepParams {
 struct ToepBars {
     uint64_t raw_full[kToepRing];
     uint64_t raw_empty[kToepRing];
-    uint64_t a_full[2];     // operand stage written by the transform
-    uint64_t a_empty[2];    // stage's output has been read by the storer
+    uint64_t a_full[2];     // A stage written by the transform
+    uint64_t a_empty[2];    // A stage's MMAs have completed
     uint64_t q_full[2];
-    uint64_t acc_full[2];
-    uint64_t acc_empty[2];
-    uint64_t out_full[2];   // stage holds the tile's output
+    uint64_t acc_full;
+    uint64_t acc_empty;
+    uint64_t out_full[2];   // buffer holds the tile's output
+    uint64_t out_empty[2];  // buffer has been read by the storer
     uint64_t fin;
     uint32_t tmem_slot;
     int abort;
@@ -179,74 +188,39 @@ __device__ __forceinline__ void build_q(uint8_t* q, const uint16_t* tst, int tid
     }
 }
 
-// Raw band layout of a half tile -> operand rows [n0, n0 + nwin) of a stage.
-// Work item = (operand row n, window row r); window rows w .. RROWS-1 are the
-// K padding of the last step and are written as zeros.  Eight consecutive
-// lanes take eight consecutive operand rows, so each quarter-warp store is
-// one 128-byte core matrix.  A warp takes two items per pass and reads both
-// before writing either, so their shared-memory loads overlap.
+// One window's rows -> its TMEM lane of an A stage: window row r at columns
+// r*RP/2 .. (r+1)*RP/2 - 1 (slot pairs), rows w .. RROWS-1 zero.
 template <int WS>
-__device__ __forceinline__ void xform_read(const uint16_t* raw, int n0, int nwin, const int* woff,
-                                           int W, int it, int nl, int rs, uint32_t (&wv)[ToepCfg<WS>::RP / 2],
-                                           uint8_t*& d0, uint8_t* dst)
+__device__ __forceinline__ void window_to_tmem(const uint16_t* src0, bool valid, int W,
+                                               uint32_t acol)
 {
     using F = ToepCfg<WS>;
-    constexpr int R4 = (F::RROWS + 3) / 4;
-    const int g8 = (n0 >> 3) + it / R4, r = (it - (it / R4) * R4) * 4 + rs;
-    const int n = g8 * 8 + nl, wn = n - n0;
-    d0 = nullptr;
-    if (r >= F::RROWS || wn < 0 || wn >= nwin)
-        return;
-    d0 = dst + g8 * F::SBO_A + (r * F::RP / 8) * 128 + nl * 16;
-    if (r >= WS) {
+#pragma unroll 2
+    for (int r = 0; r < F::RROWS; ++r) {
+        uint32_t wv[F::RP / 2];
+        if (valid && r < WS) {
+            const uint16_t* src = src0 + r * W;
+            if (WS % 2 == 0) {
 #pragma unroll
-        for (int m = 0; m < F::RP / 2; ++m)
-            wv[m] = 0u;
-        return;
-    }
-    const uint16_t* src = raw + woff[wn] + r * W;
-    if (WS % 2 == 0) {
+                for (int m = 0; m < F::RP / 2; ++m)
+                    wv[m] = (2 * m < WS) ? reinterpret_cast<const uint32_t*>(src)[m] : 0u;
+            } else {
 #pragma unroll
-        for (int m = 0; m < F::RP / 2; ++m)
-            wv[m] = (2 * m < WS) ? reinterpret_cast<const uint32_t*>(src)[m] : 0u;
-    } else {
+                for (int m = 0; m < F::RP / 2; ++m) {
+                    const uint16_t lo = (2 * m < WS) ? src[2 * m] : (uint16_t)0;
+                    const uint16_t hi = (2 * m + 1 < WS) ? src[2 * m + 1] : (uint16_t)0;
+                    wv[m] = pack_bf16x2(lo, hi);
+                }
+            }
+        } else {
 #pragma unroll
-        for (int m = 0; m < F::RP / 2; ++m) {
-            const uint16_t lo = (2 * m < WS) ? src[2 * m] : (uint16_t)0;
-            const uint16_t hi = (2 * m + 1 < WS) ? src[2 * m + 1] : (uint16_t)0;
-            wv[m] = pack_bf16x2(lo, hi);
+            for (int m = 0; m < F::RP / 2; ++m)
+                wv[m] = 0u;
         }
-    }
-}
-
-template <int WS>
-__device__ __forceinline__ void xform_write(uint8_t* d0, const uint32_t (&wv)[ToepCfg<WS>::RP / 2])
-{
-    if (d0 == nullptr)
-        return;
-#pragma unroll
-    for (int c = 0; c < ToepCfg<WS>::RP / 8; ++c)
-        *reinterpret_cast<uint4*>(d0 + c * 128) =
-            make_uint4(wv[4 * c], wv[4 * c + 1], wv[4 * c + 2], wv[4 * c + 3]);
-}
-
-template <int WS>
-__device__ __forceinline__ void transform_half(const uint16_t* raw, uint8_t* dst, int n0, int nwin,
-                                               const int* woff, int W, int tid, int nthreads)
-{
-    using F = ToepCfg<WS>;
-    constexpr int R4 = (F::RROWS + 3) / 4;
-    const int lane = tid & 31, wid = tid >> 5, nwarps = nthreads >> 5;
-    const int nl = lane & 7, rs = lane >> 3;
-    const int items = (((n0 + nwin + 7) >> 3) - (n0 >> 3)) * R4;
-    for (int it = wid; it < items; it += 2 * nwarps) {
-        uint32_t wa[F::RP / 2], wb[F::RP / 2];
-        uint8_t *da, *db = nullptr;
-        xform_read<WS>(raw, n0, nwin, woff, W, it, nl, rs, wa, da, dst);
-        if (it + nwarps < items)
-            xform_read<WS>(raw, n0, nwin, woff, W, it + nwarps, nl, rs, wb, db, dst);
-        xform_write<WS>(da, wa);
-        xform_write<WS>(db, wb);
+        if constexpr (F::RP == 16)
+            tmem_st8(acol + (uint32_t)(r * 8), wv);
+        else
+            tmem_st4(acol + (uint32_t)(r * 4), wv);
     }
 }
 
@@ -263,14 +237,14 @@ __global__ void __launch_bounds__(kToepThreads, 1)
     using F = ToepCfg<WS>;
     extern __shared__ __align__(1024) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    uint8_t* a_base = smem + P.off_a;
+    uint8_t* out_base = smem + P.off_out;
     uint8_t* q_base = smem + P.off_q;
     uint8_t* raw_base = smem + P.off_raw;
     int* woff = reinterpret_cast<int*>(smem + P.off_woff);
     uint16_t* tst = reinterpret_cast<uint16_t*>(smem + P.off_tst);
     ToepBars& S = *reinterpret_cast<ToepBars*>(smem + P.off_bar);
     volatile int* abort = &S.abort;
-    const int R = P.R;
+    const int R = P.R, NO = P.nout;
 
     // Contiguous, balanced range of items for this CTA.
     const int qn = P.items / (int)gridDim.x, rem = P.items % (int)gridDim.x;
@@ -280,16 +254,17 @@ __global__ void __launch_bounds__(kToepThreads, 1)
     if (threadIdx.x == 0) {
         for (int i = 0; i < kToepRing; ++i) {
             mbar_init(&S.raw_full[i], 1);
-            mbar_init(&S.raw_empty[i], kToepXformWarps);
+            mbar_init(&S.raw_empty[i], 4);
         }
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&S.a_full[i], kToepXformWarps);
+            mbar_init(&S.a_full[i], 4);
             mbar_init(&S.a_empty[i], 1);
             mbar_init(&S.q_full[i], kToepEpiWarps);
-            mbar_init(&S.acc_full[i], 1);
-            mbar_init(&S.acc_empty[i], kToepEpiWarps);
             mbar_init(&S.out_full[i], kToepEpiWarps);
+            mbar_init(&S.out_empty[i], 1);
         }
+        mbar_init(&S.acc_full, 1);
+        mbar_init(&S.acc_empty, kToepEpiWarps);
         mbar_init(&S.fin, 1);
         S.abort = 0;
         fence_mbar_init();
@@ -373,36 +348,33 @@ __global__ void __launch_bounds__(kToepThreads, 1)
                     cur_c = t.c;
                     ++ci;
                 }
-                const int st = seq & 1, ab = seq & 1, qb = ci & 1;
+                const int st = seq & 1, qb = ci & 1;
                 bool ok = !*abort;
                 if (first)
                     ok = ok && mbar_wait(&S.q_full[qb], (ci >> 1) & 1, abort, P.budget, P.status);
                 ok = ok && mbar_wait(&S.a_full[st], (seq >> 1) & 1, abort, P.budget, P.status);
-                if (seq >= 2)
-                    ok = ok && mbar_wait(&S.acc_empty[ab], ((seq >> 1) - 1) & 1, abort, P.budget,
-                                         P.status);
+                if (seq >= 1)
+                    ok = ok && mbar_wait(&S.acc_empty, (seq - 1) & 1, abort, P.budget, P.status);
                 if (!ok)
                     continue;
                 tc_fence_after();
-                // K step k: operand columns [16k, 16k+16) and Q rows from
-                // (w - 1 - G*k)*RP: only the start-address fields move.
+                // K step k: A columns 8k .. 8k+7 of the M tile, Q rows from
+                // (w - 1 - G*k)*RP: only the start-address field moves.
                 const uint64_t qdesc0 = smem_desc(
                     smem_u32(q_base + (size_t)qb * F::Q_BYTES) + (uint32_t)((WS - 1) * F::RP * 32),
                     128, 256);
 #pragma unroll
                 for (int mt = 0; mt < F::MTW; ++mt) {
-                    // M tile mt: windows 128*mt .. (16 groups of 8 rows further)
-                    const uint64_t adesc0 = smem_desc(
-                        smem_u32(a_base + (size_t)st * F::A_BYTES) + (uint32_t)(mt * 16) * F::SBO_A,
-                        128, F::SBO_A);
-                    const uint32_t d = tmem + (uint32_t)(ab * 256 + mt * F::DSTEP);
+                    const uint32_t a0 = tmem + (uint32_t)(st * 128 + mt * F::A_COLS);
+                    const uint32_t d = tmem + 256u + (uint32_t)(mt * F::DSTEP);
 #pragma unroll
                     for (int k = 0; k < F::KSTEPS; ++k)
-                        mma_ss(d, adesc0 + (uint64_t)(k * 16),
+                        mma_ts(d, a0 + (uint32_t)(k * 8),
                                qdesc0 - (uint64_t)(k * F::G * F::RP * 2), F::IDESC,
                                k > 0 ? 1u : 0u);
                 }
-                tc_commit(&S.acc_full[ab]);
+                tc_commit(&S.a_empty[st]);
+                tc_commit(&S.acc_full);
             }
             // Drain: all issued MMAs complete before TMEM is released.
             tc_commit(&S.fin);
@@ -411,13 +383,13 @@ __global__ void __launch_bounds__(kToepThreads, 1)
     } else if (warp == 2) {
         // ------------------------------------------------------ storer
         for (int seq = 0; seq < n_it; ++seq) {
-            const int st = seq & 1;
+            const int ob = seq % NO;
             bool ok = !*abort;
-            ok = ok && mbar_wait(&S.out_full[st], (seq >> 1) & 1, abort, P.budget, P.status);
+            ok = ok && mbar_wait(&S.out_full[ob], (seq / NO) & 1, abort, P.budget, P.status);
             ok = __all_sync(0xffffffffu, ok);
             if (ok) {
                 const BandTile t = toep_tile(P, it0 + seq);
-                const uint8_t* out = a_base + (size_t)st * F::A_BYTES;
+                const uint8_t* out = out_base + (size_t)ob * F::OUT_BYTES;
                 if (P.use_tmap) {
                     // planes past the last image are clipped
                     if (lane == 0)
@@ -436,39 +408,51 @@ __global__ void __launch_bounds__(kToepThreads, 1)
             }
             __syncwarp();
             if (ok && lane == 0)
-                mbar_arrive(&S.a_empty[st]);
+                mbar_arrive(&S.out_empty[ob]);
         }
         bulk_wait<0>();
     } else if (warp < kToepEpiWarp0) {
         // ------------------------------------------------------ transform
-        const int tt = threadIdx.x - kToepXformWarp0 * 32;
+        // Thread = window mt*128 + quarter*32 + lane.  tcgen05.st writes all
+        // 32 lanes of the quarter, so a tile is written once both halves
+        // have landed.
+        const int quarter = warp & 3;
+        const uint32_t lanebase = (uint32_t)(quarter * 32) << 16;
         for (int seq = 0; seq < n_it; ++seq) {
             const BandTile t = toep_tile(P, it0 + seq);
             const int st = seq & 1;
-            uint8_t* stage = a_base + (size_t)st * F::A_BYTES;
             bool ok = !*abort;
             if (seq >= 2)
                 ok = ok && mbar_wait(&S.a_empty[st], ((seq >> 1) - 1) & 1, abort, P.budget,
                                      P.status);
-            for (int h = 0; h < 2; ++h) {
-                const int ss = 2 * seq + h, s = ss % R;
-                ok = ok && mbar_wait(&S.raw_full[s], (ss / R) & 1, abort, P.budget, P.status);
-                ok = __all_sync(0xffffffffu, ok);
-                if (ok) {
-                    const BandTile sh = toep_half(P, t, h);
-                    const uint16_t* raw =
-                        reinterpret_cast<const uint16_t*>(raw_base + (size_t)s * P.sub_bytes);
-                    transform_half<WS>(raw, stage, h * P.sb * P.nw, sh.nb * P.nw, woff, P.W, tt,
-                                       kToepXformWarps * 32);
+            const int ss0 = 2 * seq, s0 = ss0 % R, s1 = (ss0 + 1) % R;
+            ok = ok && mbar_wait(&S.raw_full[s0], (ss0 / R) & 1, abort, P.budget, P.status);
+            ok = ok && mbar_wait(&S.raw_full[s1], ((ss0 + 1) / R) & 1, abort, P.budget, P.status);
+            ok = __all_sync(0xffffffffu, ok);
+            tc_fence_after();
+            if (ok) {
+                const int nwin = t.nb * P.nw;
+                const int h0win = toep_half(P, t, 0).nb * P.nw;
+#pragma unroll 1
+                for (int mt = 0; mt < F::MTW; ++mt) {
+                    const int n = mt * 128 + quarter * 32 + lane;
+                    const bool valid = n < nwin;
+                    const int h = n < h0win ? 0 : 1;
+                    const uint16_t* raw = reinterpret_cast<const uint16_t*>(
+                        raw_base + (size_t)(h ? s1 : s0) * P.sub_bytes);
+                    const uint16_t* src0 = raw + (valid ? woff[h ? n - h0win : n] : 0);
+                    window_to_tmem<WS>(src0, valid, P.W,
+                                       tmem + lanebase + (uint32_t)(st * 128 + mt * F::A_COLS));
                 }
-                __syncwarp();
-                if (ok && lane == 0)
-                    mbar_arrive(&S.raw_empty[s]);
+                tmem_wait_st();
             }
-            fence_proxy_async_smem();
+            tc_fence_before();
             __syncwarp();
-            if (ok && lane == 0)
+            if (ok && lane == 0) {
+                mbar_arrive(&S.raw_empty[s0]);
+                mbar_arrive(&S.raw_empty[s1]);
                 mbar_arrive(&S.a_full[st]);
+            }
         }
     } else {
         // ------------------------------------------------------ epilogue
@@ -499,54 +483,57 @@ __global__ void __launch_bounds__(kToepThreads, 1)
         for (int seq = 0; seq < n_it; ++seq) {
             const BandTile t = toep_tile(P, it0 + seq);
             const int nwin = t.nb * P.nw;
-            const int ab = seq & 1, st = seq & 1;
+            const int ob = seq % NO;
             bool ok = !*abort;
-            ok = ok && mbar_wait(&S.acc_full[ab], (seq >> 1) & 1, abort, P.budget, P.status);
+            ok = ok && mbar_wait(&S.acc_full, seq & 1, abort, P.budget, P.status);
+            if (seq >= NO)
+                ok = ok && mbar_wait(&S.out_empty[ob], ((seq / NO) - 1) & 1, abort, P.budget,
+                                     P.status);
             ok = __all_sync(0xffffffffu, ok);
             tc_fence_after();
+            uint16_t* obuf = reinterpret_cast<uint16_t*>(out_base + (size_t)ob * F::OUT_BYTES);
 #pragma unroll 1
             for (int mt = 0; mt < F::MTW; ++mt) {
-              const int n = mt * 128 + quarter * 32 + lane;
-              if (ok && mt * 128 + quarter * 32 < nwin) {
+                const int n = mt * 128 + quarter * 32 + lane;
+                if (!ok || mt * 128 + quarter * 32 >= nwin)
+                    continue;
                 const bool valid = n < nwin;
-                uint16_t* o0 = reinterpret_cast<uint16_t*>(a_base + (size_t)st * F::A_BYTES) +
-                               (valid ? woff[n] : 0);
-                const uint32_t lrow = tmem + ((uint32_t)(quarter * 32) << 16) +
-                                      (uint32_t)(ab * 256 + mt * F::DSTEP);
+                uint16_t* o0 = obuf + (valid ? woff[n] : 0);
+                const uint32_t lrow = tmem + ((uint32_t)(quarter * 32) << 16) + 256u +
+                                      (uint32_t)(mt * F::DSTEP);
 #pragma unroll 1
                 for (int li = hf; li < F::LOADS; li += 2) {
                     uint32_t r[32];
                     tmem_ld32(lrow + (uint32_t)(li * 32), r);
                     tmem_wait_ld(r);
-                    if (valid) {
+                    if (!valid)
+                        continue;
 #pragma unroll
-                        for (int rr = 0; rr < F::RL; ++rr) {
-                            const int pr = li * F::RL + rr;
-                            if (pr < WS) {
-                                uint16_t* o = o0 + pr * P.W;
-                                if (WS % 2 == 0) {
+                    for (int rr = 0; rr < F::RL; ++rr) {
+                        const int pr = li * F::RL + rr;
+                        if (pr >= WS)
+                            continue;
+                        uint16_t* o = o0 + pr * P.W;
+                        if (WS % 2 == 0) {
 #pragma unroll
-                                    for (int m = 0; m < WS / 2; ++m)
-                                        reinterpret_cast<uint32_t*>(o)[m] = bf16x2_rn(
-                                            r[rr * F::RP + 2 * m], r[rr * F::RP + 2 * m + 1]);
-                                } else {
+                            for (int m = 0; m < WS / 2; ++m)
+                                reinterpret_cast<uint32_t*>(o)[m] =
+                                    bf16x2_rn(r[rr * F::RP + 2 * m], r[rr * F::RP + 2 * m + 1]);
+                        } else {
 #pragma unroll
-                                    for (int s = 0; s < WS; ++s)
-                                        o[s] = __bfloat16_as_ushort(__float2bfloat16_rn(
-                                            __uint_as_float(r[rr * F::RP + s])));
-                                }
-                            }
+                            for (int s = 0; s < WS; ++s)
+                                o[s] = __bfloat16_as_ushort(
+                                    __float2bfloat16_rn(__uint_as_float(r[rr * F::RP + s])));
                         }
                     }
                 }
-              }
             }
             tc_fence_before();
             fence_proxy_async_smem();
             __syncwarp();
             if (ok && lane == 0) {
-                mbar_arrive(&S.acc_empty[ab]);
-                mbar_arrive(&S.out_full[st]);
+                mbar_arrive(&S.acc_empty);
+                mbar_arrive(&S.out_full[ob]);
             }
             if (t.c != cur_c) {
                 cur_c = t.c;
@@ -575,24 +562,28 @@ constexpr uint32_t kMinSmem = 120 * 1024;
 inline uint32_t align_up(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
 
 struct ToepLayout {
-    uint32_t off_a, off_q, off_raw, off_woff, off_bar, off_tst, total, sub_bytes;
-    int R, bpt, sb;
+    uint32_t off_out, off_q, off_raw, off_woff, off_bar, off_tst, total, sub_bytes;
+    int R, bpt, sb, nout;
 };
 
+// Q (two channels) | output buffers | window offsets | staged table |
+// barriers | raw ring.  Two output buffers when the ring still gets at least
+// four half tiles, else one.
 template <int WS>
-bool toep_layout(const Geom& g, ToepLayout& L)
+bool toep_layout_n(const Geom& g, int nout, ToepLayout& L)
 {
     using F = ToepCfg<WS>;
     if (g.nw < 1 || g.nw > F::TW)
         return false;
+    L.nout = nout;
     L.bpt = F::TW / g.nw;
     L.sb = (L.bpt + 1) / 2;
     L.sub_bytes = align_up((uint32_t)L.sb * WS * g.W * 2, 128);
     uint32_t off = 0;
-    L.off_a = off;                                   // 1024-aligned stages
-    off += 2 * F::A_BYTES;
-    L.off_q = align_up(off, 128);
-    off = L.off_q + 2 * F::Q_BYTES;
+    L.off_q = off;
+    off += 2 * F::Q_BYTES;
+    L.off_out = align_up(off, 128);
+    off = L.off_out + (uint32_t)nout * F::OUT_BYTES;
     L.off_woff = align_up(off, 16);
     off = L.off_woff + F::TW * 4;
     L.off_tst = align_up(off, 16);
@@ -614,6 +605,14 @@ bool toep_layout(const Geom& g, ToepLayout& L)
     if (L.total < kMinSmem)
         L.total = kMinSmem;
     return L.total <= kSmemMax;
+}
+
+template <int WS>
+bool toep_layout(const Geom& g, ToepLayout& L)
+{
+    if (toep_layout_n<WS>(g, 2, L) && L.R >= 4)
+        return true;
+    return toep_layout_n<WS>(g, 1, L);
 }
 
 template <int WS, int MODE>
@@ -654,7 +653,8 @@ cudaError_t toep_launch_ws(const Geom& g, const void* x, const void* T, void* y,
             P.kimg_sub = ks;
         }
     }
-    P.off_a = lay.off_a; P.off_q = lay.off_q; P.off_raw = lay.off_raw;
+    P.nout = lay.nout;
+    P.off_out = lay.off_out; P.off_q = lay.off_q; P.off_raw = lay.off_raw;
     P.off_woff = lay.off_woff; P.off_bar = lay.off_bar; P.off_tst = lay.off_tst;
     P.budget = L.budget;
     P.status = L.status;
