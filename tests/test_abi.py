@@ -75,6 +75,8 @@ def test_workspace_size_formula(lib):
     assert f(64, 128, 56, 56, 14, 1) == tc(128 + 255)
     # 32 images of 112x112: 8 bands/tile, 32 tiles/channel, 128 tiles
     assert f(32, 4, 112, 112, 14, 1) == tc(4 + 127)
+    # 2 images of 112x112, w = 7: 64-window tiles of 4 bands, 8 tiles/channel
+    assert f(2, 4, 112, 112, 7, 1) == tc(4 + 31, 169)
     # fp32, CUDA-core path: chunks of 8 bands per channel
     assert f(2, 3, 14, 28, 7, 0) == 3 * 1 * 169 * 4
     assert f(1, 1, 14, 15, 7, 1) == 0

@@ -88,51 +88,87 @@ __device__ __forceinline__ void band_run(const BandTile& t, const BandRuns& R, i
 
 // Raw band layout -> operand tile with rows = windows n (8-row groups
 // `sbo` bytes apart) and columns = padded positions (core matrices of 8
-// slots, 128 bytes apart).  Work item = (window n, window row r); one thread
-// reads the row and writes RP/8 16-byte core-matrix rows.  Eight consecutive
-// lanes take eight consecutive windows, so each quarter-warp store is one
-// contiguous 128-byte line.  Rows nwin <= n < nzero are written as zeros;
-// rows past that are left as they are.
+// slots, 128 bytes apart).  A warp takes one group of eight windows: lane
+// (nl, rs) handles window 8*g + nl and window rows rs, rs + 4, ...; all of a
+// lane's rows are read before any is written, so its loads overlap.  Eight
+// consecutive lanes take eight consecutive windows, so each quarter-warp
+// store is one contiguous 128-byte line.  Rows nwin <= n < nend are written
+// as zeros; rows past that are left as they are.
 template <int WS>
-__device__ __forceinline__ void transform_rows(const uint16_t* raw, uint8_t* dst, uint32_t sbo,
-                                               int nwin, int nzero, const int* woff, int W,
-                                               int tid, int nthreads)
+__device__ __forceinline__ void transform_group(const uint16_t* raw, uint8_t* dst, uint32_t sbo,
+                                                int g8, int nwin, int nend, const int* woff,
+                                                int W, int lane)
 {
     using P = PadCfg<WS>;
     constexpr int R4 = (WS + 3) / 4;
-    const int lane = tid & 31, wid = tid >> 5, nwarps = nthreads >> 5;
     const int nl = lane & 7, rs = lane >> 3;
-    const int nend = nzero > nwin ? nzero : nwin;
-    const int groups = (nend + 7) >> 3;
-    for (int it = wid; it < groups * R4; it += nwarps) {
-        const int g8 = it / R4, r = (it - g8 * R4) * 4 + rs;
-        const int n = g8 * 8 + nl;
-        if (r >= WS || n >= nend)
-            continue;
-        const uint16_t* src = raw + woff[n < nwin ? n : 0] + r * W;
-        uint8_t* d0 = dst + g8 * sbo + (r * P::RP / 8) * 128 + nl * 16;
-        uint32_t wv[P::RP / 2];
-        if (n >= nwin) {
+    const int n = g8 * 8 + nl;
+    if (n >= nend)
+        return;
+    const uint16_t* base = raw + woff[n < nwin ? n : 0];
+    uint32_t wv[R4][P::RP / 2];
+#pragma unroll
+    for (int q = 0; q < R4; ++q) {
+        const int r = q * 4 + rs;
+        const uint16_t* src = base + r * W;
+        if (n >= nwin || r >= WS) {
 #pragma unroll
             for (int m = 0; m < P::RP / 2; ++m)
-                wv[m] = 0u;
+                wv[q][m] = 0u;
         } else if (WS % 2 == 0) {
 #pragma unroll
             for (int m = 0; m < P::RP / 2; ++m)
-                wv[m] = (2 * m < WS) ? reinterpret_cast<const uint32_t*>(src)[m] : 0u;
+                wv[q][m] = (2 * m < WS) ? reinterpret_cast<const uint32_t*>(src)[m] : 0u;
         } else {
 #pragma unroll
             for (int m = 0; m < P::RP / 2; ++m) {
                 const uint16_t lo = (2 * m < WS) ? src[2 * m] : (uint16_t)0;
                 const uint16_t hi = (2 * m + 1 < WS) ? src[2 * m + 1] : (uint16_t)0;
-                wv[m] = pack_bf16x2(lo, hi);
+                wv[q][m] = pack_bf16x2(lo, hi);
             }
         }
+    }
+    uint8_t* d0 = dst + g8 * sbo + nl * 16;
 #pragma unroll
-        for (int c = 0; c < P::RP / 8; ++c) {
-            uint4 v = make_uint4(wv[4 * c], wv[4 * c + 1], wv[4 * c + 2], wv[4 * c + 3]);
-            *reinterpret_cast<uint4*>(d0 + c * 128) = v;
-        }
+    for (int q = 0; q < R4; ++q) {
+        const int r = q * 4 + rs;
+        if (r >= WS)
+            continue;
+#pragma unroll
+        for (int c = 0; c < P::RP / 8; ++c)
+            *reinterpret_cast<uint4*>(d0 + (r * P::RP / 8 + c) * 128) =
+                make_uint4(wv[q][4 * c], wv[q][4 * c + 1], wv[q][4 * c + 2], wv[q][4 * c + 3]);
+    }
+}
+
+// One tile: windows [0, nwin), zero rows up to nzero.  Warps take groups.
+template <int WS>
+__device__ __forceinline__ void transform_rows(const uint16_t* raw, uint8_t* dst, uint32_t sbo,
+                                               int nwin, int nzero, const int* woff, int W,
+                                               int tid, int nthreads)
+{
+    const int lane = tid & 31, wid = tid >> 5, nwarps = nthreads >> 5;
+    const int nend = nzero > nwin ? nzero : nwin;
+    const int groups = (nend + 7) >> 3;
+    for (int g8 = wid; g8 < groups; g8 += nwarps)
+        transform_group<WS>(raw, dst, sbo, g8, nwin, nend, woff, W, lane);
+}
+
+// Two tiles of the same windows (from two tensors) in one pass: warps take
+// the groups of both, so small tiles still keep every warp busy.
+template <int WS>
+__device__ __forceinline__ void transform_rows_pair(const uint16_t* raw0, uint8_t* dst0,
+                                                    const uint16_t* raw1, uint8_t* dst1,
+                                                    uint32_t sbo, int nwin, int nzero,
+                                                    const int* woff, int W, int tid, int nthreads)
+{
+    const int lane = tid & 31, wid = tid >> 5, nwarps = nthreads >> 5;
+    const int nend = nzero > nwin ? nzero : nwin;
+    const int groups = (nend + 7) >> 3;
+    for (int it = wid; it < 2 * groups; it += nwarps) {
+        const bool second = it >= groups;
+        transform_group<WS>(second ? raw1 : raw0, second ? dst1 : dst0, sbo,
+                            second ? it - groups : it, nwin, nend, woff, W, lane);
     }
 }
 

@@ -45,7 +45,7 @@
 namespace wbmm {
 
 constexpr uint32_t kSmemMax = 232448;
-constexpr int kDtRing = 2;
+constexpr int kDtRingMax = 8;
 constexpr int kDtXformWarps = 8;                 // warps 2..9
 constexpr int kDtEpiWarp0 = 2 + kDtXformWarps;  // warps 10..17
 constexpr int kDtEpiWarps = 8;
@@ -71,19 +71,10 @@ constexpr uint32_t dt_stg_bytes(int ws)
     return (uint32_t)(128 / ((ws + 7) / 8 * 8)) * dt_stg_stride(ws) * 4;
 }
 
-// Shared memory of the dT kernel for window size ws and nt windows per tile:
-// two operand stages (dY and x tiles), the raw ring, the staging array,
-// barriers.
-constexpr uint32_t dt_smem_bytes(int ws, int nt)
-{
-    const int d = ws * ws, rp = (ws + 7) / 8 * 8, kp = (ws * rp + 15) / 16 * 16;
-    const uint32_t stage = 2u * (uint32_t)nt * kp * 2;
-    const uint32_t raw = 2u * (uint32_t)((nt * d * 2 + 127) / 128 * 128);
-    return 2 * stage + kDtRing * raw + dt_stg_bytes(ws) + nt * 4 + 2048;
-}
-
-// Windows per tile: 64 when the layout fits, else 32 (w >= 15).
-constexpr int dt_nt_for(int ws) { return dt_smem_bytes(ws, 64) <= kSmemMax ? 64 : 32; }
+// Windows per tile (the MMA K of one stage): 64, or 32 for w = 16 where two
+// 64-window stages and two raw slots do not fit.  (Measured at w = 14: 32-
+// window tiles with a six-deep ring run ~10% slower than 64-window tiles.)
+constexpr int dt_nt_for(int ws) { return ws >= 15 ? 32 : 64; }
 
 template <int WS>
 struct DtCfg : PadCfg<WS> {
@@ -119,14 +110,15 @@ struct TcDtParams {
                             // reads and writes nothing it touches
     int use_tmap;           // tiles are whole planes: one 4-D TMA per tensor
     int kimg;               // planes per tile when use_tmap
+    int R;                  // raw ring depth (tiles)
     uint32_t off_raw, off_stage, off_stg, off_woff, off_bar;
     unsigned long long budget;
     int* status;
 };
 
 struct DtBars {
-    uint64_t raw_full[kDtRing];
-    uint64_t raw_empty[kDtRing];
+    uint64_t raw_full[kDtRingMax];
+    uint64_t raw_empty[kDtRingMax];
     uint64_t st_full[2];
     uint64_t st_empty[2];
     uint64_t g_full;
@@ -135,6 +127,7 @@ struct DtBars {
     uint32_t tmem_slot;
     int abort;
     int seg_ok;             // the later segments of the current channel arrived
+    int pre_ok;             // ... and did so before its reduction began
 };
 
 struct DtTile {
@@ -195,7 +188,7 @@ __global__ void __launch_bounds__(kDtThreads, 1) wbmm_tc_dt_kernel(const __grid_
     volatile int* abort = &S.abort;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kDtRing; ++i) {
+        for (int i = 0; i < kDtRingMax; ++i) {
             mbar_init(&S.raw_full[i], 1);
             mbar_init(&S.raw_empty[i], kDtXformWarps);
         }
@@ -241,10 +234,10 @@ __global__ void __launch_bounds__(kDtThreads, 1) wbmm_tc_dt_kernel(const __grid_
         int issued = 0, seq = 0;
         DtWalker it;
         for (it.start(P); it.valid(P); it.next(P), ++seq) {
-            const int s = seq % kDtRing;
+            const int s = seq % P.R;
             bool ok = !*abort;
-            if (seq >= kDtRing)
-                ok = ok && mbar_wait(&S.raw_empty[s], ((seq / kDtRing) - 1) & 1, abort, P.budget,
+            if (seq >= P.R)
+                ok = ok && mbar_wait(&S.raw_empty[s], ((seq / P.R) - 1) & 1, abort, P.budget,
                                      P.status);
             if (!__all_sync(0xffffffffu, ok))
                 break;
@@ -274,9 +267,9 @@ __global__ void __launch_bounds__(kDtThreads, 1) wbmm_tc_dt_kernel(const __grid_
             issued = seq + 1;
         }
         if (lane == 0) {
-            for (int s = 0; s < kDtRing && s < issued; ++s) {
-                const int last = s + ((issued - 1 - s) / kDtRing) * kDtRing;
-                mbar_wait_drain(&S.raw_full[s], (last / kDtRing) & 1, P.budget, P.status);
+            for (int s = 0; s < P.R && s < issued; ++s) {
+                const int last = s + ((issued - 1 - s) / P.R) * P.R;
+                mbar_wait_drain(&S.raw_full[s], (last / P.R) & 1, P.budget, P.status);
             }
         }
     } else if (warp == 1) {
@@ -339,9 +332,9 @@ __global__ void __launch_bounds__(kDtThreads, 1) wbmm_tc_dt_kernel(const __grid_
         DtWalker it;
         for (it.start(P); it.valid(P); it.next(P), ++seq) {
             const DtTile t = it.get(P);
-            const int s = seq % kDtRing, bs = seq & 1;
+            const int s = seq % P.R, bs = seq & 1;
             bool ok = !*abort;
-            ok = ok && mbar_wait(&S.raw_full[s], (seq / kDtRing) & 1, abort, P.budget, P.status);
+            ok = ok && mbar_wait(&S.raw_full[s], (seq / P.R) & 1, abort, P.budget, P.status);
             if (seq >= 2)
                 ok = ok && mbar_wait(&S.st_empty[bs], ((seq >> 1) - 1) & 1, abort, P.budget,
                                      P.status);
@@ -352,10 +345,9 @@ __global__ void __launch_bounds__(kDtThreads, 1) wbmm_tc_dt_kernel(const __grid_
                 uint8_t* stage = st_base + (size_t)bs * F::STAGE_BYTES;
                 const int nwin = t.bt.nb * P.nw;
                 const int nzero = (nwin + 15) & ~15;    // last MMA K step reads up to here
-                transform_rows<WS>(raw, stage, F::SBO_T, nwin, nzero, woff, P.W, tt,
-                                   kDtXformWarps * 32);
-                transform_rows<WS>(raw + F::RAW_HALF / 2, stage + F::TILE_BYTES, F::SBO_T, nwin,
-                                   nzero, woff, P.W, tt, kDtXformWarps * 32);
+                transform_rows_pair<WS>(raw, stage, raw + F::RAW_HALF / 2, stage + F::TILE_BYTES,
+                                        F::SBO_T, nwin, nzero, woff, P.W, tt,
+                                        kDtXformWarps * 32);
                 fence_proxy_async_smem();
             }
             __syncwarp();
@@ -396,6 +388,40 @@ __global__ void __launch_bounds__(kDtThreads, 1) wbmm_tc_dt_kernel(const __grid_
             ok = ok && mbar_wait(&S.g_full, item_seq & 1, abort, P.budget, P.status);
             ok = __all_sync(0xffffffffu, ok);
             tc_fence_after();
+            const int k = (int)blockIdx.x;
+            const int k0 = dt_cta_of(P, (long long)c * P.tpc);
+            const int k1 = dt_cta_of(P, (long long)c * P.tpc + P.tpc - 1);
+            // The channel's first tiles and last segment: the later segments
+            // (one or two CTAs) were normally published long ago, so their
+            // partial sums are fetched now and arrive during the reduction.
+            const bool gather = k == k0 && k1 > k0 && k1 - k0 <= 2;
+            float pre[2][NBT];
+            bool pre_ok = false;
+            if (gather) {
+                if (et == 0) {
+                    int r = 1;
+                    for (int kk = k0 + 1; kk <= k1; ++kk)
+                        r &= ld_acquire_u64(P.flags + c + kk) == P.token ? 1 : 0;
+                    S.pre_ok = r;
+                }
+                named_bar_sync(3, kDtEpiThreads);
+                pre_ok = S.pre_ok != 0;
+                named_bar_sync(3, kDtEpiThreads);   // pre_ok is rewritten next
+                if (pre_ok && ok) {
+                    __threadfence();
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+#pragma unroll
+                        for (int i = 0; i < NBT; ++i) {
+                            const int bin = et + i * kDtEpiThreads;
+                            pre[j][i] = (k0 + 1 + j <= k1 && bin < F::TSZ)
+                                            ? __ldcg(P.partials +
+                                                     (long long)(c + k0 + 1 + j) * F::TSZ + bin)
+                                            : 0.0f;
+                        }
+                    }
+                }
+            }
             float acc[NBT];
 #pragma unroll
             for (int i = 0; i < NBT; ++i)
@@ -420,7 +446,7 @@ __global__ void __launch_bounds__(kDtThreads, 1) wbmm_tc_dt_kernel(const __grid_
                         for (int b = 0; b < NB; ++b) {
                             const int rr = ch * NB + b;
                             if (rr < WS) {
-                                float a = 0.0f, c = 0.0f;
+                                float a = 0.0f, wrap = 0.0f;
 #pragma unroll
                                 for (int s = 0; s < WS; ++s) {
                                     const float g = __shfl_sync(0xffffffffu, v[b * RP + s],
@@ -428,11 +454,11 @@ __global__ void __launch_bounds__(kDtThreads, 1) wbmm_tc_dt_kernel(const __grid_
                                     if (L + s < RP)
                                         a += g;
                                     else
-                                        c += g;
+                                        wrap += g;
                                 }
                                 float* row = stg + ((ubase - mt * 128 + lane) / RP) * SP + rr * 2 * RP;
                                 row[L + RP] = a;
-                                row[L] = c;
+                                row[L] = wrap;
                             }
                         }
                     }
@@ -470,8 +496,6 @@ __global__ void __launch_bounds__(kDtThreads, 1) wbmm_tc_dt_kernel(const __grid_
                 }
                 named_bar_sync(3, kDtEpiThreads);
             }
-            const int k0 = dt_cta_of(P, (long long)c * P.tpc);
-            const int k1 = dt_cta_of(P, (long long)c * P.tpc + P.tpc - 1);
             if (k0 == k1) {
                 // the whole channel is in this CTA's range
                 if (ok) {
@@ -485,7 +509,6 @@ __global__ void __launch_bounds__(kDtThreads, 1) wbmm_tc_dt_kernel(const __grid_
                 }
                 continue;
             }
-            const int k = (int)blockIdx.x;
             if (k != k0) {
                 // an earlier segment of this CTA: publish it for CTA k0
                 float* out = P.partials + (long long)(c + k) * F::TSZ;
@@ -502,7 +525,23 @@ __global__ void __launch_bounds__(kDtThreads, 1) wbmm_tc_dt_kernel(const __grid_
                 continue;
             }
             // this CTA holds the channel's first tiles and its last segment:
-            // wait for the later segments, then add them in CTA order
+            // add the later segments in CTA order
+            if (pre_ok) {
+                if (ok) {
+#pragma unroll
+                    for (int i = 0; i < NBT; ++i) {
+                        const int bin = et + i * kDtEpiThreads;
+                        if (bin < F::TSZ) {
+                            float sum = acc[i] + pre[0][i];
+                            if (k1 - k0 == 2)
+                                sum += pre[1][i];
+                            P.dT[(long long)c * F::TSZ + bin] = sum;
+                        }
+                    }
+                }
+                continue;
+            }
+            // otherwise wait for them first
             if (et == 0) {
                 int good = 1;
                 for (int kk = k0 + 1; kk <= k1 && good; ++kk)
@@ -545,8 +584,11 @@ inline uint32_t align_up(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
 
 struct DtLayout {
     uint32_t off_raw, off_stage, off_stg, off_woff, off_bar, total;
+    int R;
 };
 
+// Operand stages | staging array | window offsets | barriers | raw ring,
+// as many raw slots as fit (at most kDtRingMax).
 template <int WS>
 DtLayout dt_layout()
 {
@@ -555,14 +597,17 @@ DtLayout dt_layout()
     uint32_t off = 0;
     L.off_stage = off;
     off += 2 * F::STAGE_BYTES;
-    L.off_raw = align_up(off, 128);
-    off = L.off_raw + kDtRing * F::RAW_BYTES;
     L.off_stg = align_up(off, 16);
     off = L.off_stg + dt_stg_bytes(WS);
     L.off_woff = align_up(off, 16);
     off = L.off_woff + F::NT * 4;
     L.off_bar = align_up(off, 16);
     off = L.off_bar + sizeof(DtBars);
+    L.off_raw = align_up(off, 128);
+    const uint32_t avail = kSmemMax - 1024 > L.off_raw ? kSmemMax - 1024 - L.off_raw : 0;
+    int R = (int)(avail / F::RAW_BYTES);
+    L.R = R < kDtRingMax ? R : kDtRingMax;
+    off = L.off_raw + (uint32_t)L.R * F::RAW_BYTES;
     L.total = align_up(off, 1024);
     // at least half the SM's shared memory: one CTA (and one 512-column TMEM
     // allocation) per SM
@@ -618,7 +663,7 @@ cudaError_t dt_launch_ws(const Geom& g, const void* x, const void* dy, float* wo
 {
     using F = DtCfg<WS>;
     const DtLayout lay = dt_layout<WS>();
-    if (lay.total > kSmemMax)
+    if (lay.total > kSmemMax || lay.R < 2)
         return cudaErrorInvalidConfiguration;
     static unsigned long long configured = 0;
     int dev = 0;
@@ -660,6 +705,7 @@ cudaError_t dt_launch_ws(const Geom& g, const void* x, const void* dy, float* wo
             P.kimg = k;
         }
     }
+    P.R = lay.R;
     P.off_raw = lay.off_raw; P.off_stage = lay.off_stage; P.off_stg = lay.off_stg;
     P.off_woff = lay.off_woff; P.off_bar = lay.off_bar;
     P.budget = L.budget;
