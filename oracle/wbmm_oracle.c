@@ -171,7 +171,6 @@ void oracle_reparam_merge(const double *Tw, const double *Tk, double *M, int C, 
 }
 
 /*
- * Inter-block 3x3 depthwise mixing (reading notes, "Method", third point):/*
  * Inter-block 3x3 depthwise mixing (reading notes, "Method", third point):
  * z[b,c,h,x] = sum_{a,e in 0..2} K[c,a,e] * y[b,c,h+a-1,x+e-1], with y taken
  * as zero outside the image (cross-correlation, zero padding 1, no bias).

@@ -17,9 +17,13 @@ def declared_symbols():
 
 @pytest.fixture(scope="module")
 def lib():
-    from windowed_matmul_conv_b200 import build
-    path = build.build()
-    return ctypes.CDLL(path)
+    # by path: the package's __init__ refuses to import before the library exists
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "_wbmm_build", os.path.join(ROOT, "windowed_matmul_conv_b200", "build.py"))
+    build = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(build)
+    return ctypes.CDLL(build.build())
 
 
 def test_header_declares_the_entry_points():
