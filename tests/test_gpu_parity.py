@@ -307,7 +307,9 @@ def test_fused_cached_dw3x3_unsupported_shapes():
 
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
-@pytest.mark.parametrize("hw", [(37, 70), (40, 64), (33, 8)])  # scalar and 16-byte-row paths
+# scalar path (W % 8 != 0) and the 16-byte-vector path: one vector per row,
+# one 32-vector chunk, several chunks with a ragged last one, a single row
+@pytest.mark.parametrize("hw", [(37, 70), (40, 64), (33, 8), (19, 264), (9, 520), (1, 16)])
 def test_dw3x3(dtype, hw):
     y = gen((3, 4) + hw, 16, dtype)
     K = gen((4, 1, 3, 3), 17, dtype, 1.0 / 3.0)

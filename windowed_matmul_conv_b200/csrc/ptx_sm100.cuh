@@ -170,6 +170,28 @@ __device__ __forceinline__ void cp_async_wait_all()
     asm volatile("cp.async.wait_all;" ::: "memory");
 }
 
+// Global -> shared copy of 16 bytes (both addresses 16-byte aligned) that
+// reads src_bytes (0 or 16) from gsrc and zero-fills the rest; one commit
+// group per call of cp_async_commit, completed in order.
+__device__ __forceinline__ void cp_async_16z(uint32_t smem_dst, const void *gsrc, uint32_t src_bytes)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_dst), "l"(gsrc),
+                 "r"(src_bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void cp_async_commit()
+{
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+// Waits until at most N of this thread's most recent commit groups are pending.
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group()
+{
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // ------------------------------------------------------- bulk async copies
 // Global -> shared, completion signalled on `bar` as transaction bytes.
 // Both addresses 16-byte aligned, bytes a multiple of 16.

@@ -317,50 +317,104 @@ __global__ void dw3x3_kernel(const TIn* __restrict__ y, const TIn* __restrict__ 
     }
 }
 
-// bf16 maps whose rows are whole 16-byte vectors (W % 8 == 0): a band of
-// kDwVecRows output rows plus one halo row above and below is staged in
-// shared memory with 16-byte loads; each thread makes 8 consecutive outputs
-// and writes them as one 16-byte store.  Same fp32 fused multiply-add order
-// as dw3x3_kernel (a outer, e inner, zero padding included), so both kernels
-// give the same bits.
-constexpr int kDwVecRows = 16;
+// bf16 maps whose rows are whole 16-byte vectors (W % 8 == 0), streamed.
+// Lane = one 16-byte vector of a 32-vector chunk (256 columns) of a plane; a
+// warp walks down rows.  The flattened row space (plane-chunk, row) is cut
+// into one contiguous, balanced range per warp, so every warp streams the
+// same number of rows.  Each lane keeps its own column of the next kDwRing
+// input rows in flight with 16-byte asynchronous copies into a ring in shared
+// memory (rows outside the image are zero-filled by the copy); a row is read
+// back once, unpacked into fp32 pairs (its left and right neighbour values
+// from the adjacent lanes by shuffles, or a 2-byte load at a chunk edge inside
+// the row), and its slot is refilled at once.  The three live rows stay
+// unpacked in registers.  The per-output arithmetic is dw3x3_pairs8, as in
+// every other bf16 3x3 path, so all of them give the same bits.
+constexpr int kDwRing = 16;
+constexpr int kDwWarps = 4;
+constexpr int kDwBlocksPerSm = 4;
+constexpr size_t kDwSmem = (size_t)kDwWarps * kDwRing * 32 * 16;
 
-__global__ void __launch_bounds__(256) dw3x3_bf16_vec_kernel(const uint16_t* __restrict__ y,
-                                                             const uint16_t* __restrict__ K,
-                                                             uint16_t* __restrict__ z, int C,
-                                                             int H, int W, int tiles_y)
+__global__ void __launch_bounds__(kDwWarps * 32, kDwBlocksPerSm) dw3x3_bf16_rows_kernel(
+    const uint16_t* __restrict__ y, const uint16_t* __restrict__ K, uint16_t* __restrict__ z,
+    int C, int H, int W, int chunks, long long total_rows)
 {
+    extern __shared__ uint4 dw_ring[];
     grid_dep_wait();
     grid_dep_launch();
-    extern __shared__ uint4 sband[];
+    const int lane = threadIdx.x & 31;
+    const uint32_t ring0 = smem_u32(dw_ring + (threadIdx.x >> 5) * kDwRing * 32 + lane);
+    const uint4* ringp = dw_ring + (threadIdx.x >> 5) * kDwRing * 32 + lane;
+    const long long gw = (long long)blockIdx.x * kDwWarps + (threadIdx.x >> 5);
+    const long long nwarps = (long long)gridDim.x * kDwWarps;
+    const long long qn = total_rows / nwarps, rem = total_rows % nwarps;
+    long long r = gw * qn + (gw < rem ? gw : rem);
+    const long long r1 = r + qn + (gw < rem ? 1 : 0);
     const int nvec = W / 8;
-    const long long bc = blockIdx.x / tiles_y;
-    const int ty = blockIdx.x - (int)(bc * tiles_y);
-    const int c = (int)(bc % C);
-    const int h0 = ty * kDwVecRows;
-    const uint4* yp = reinterpret_cast<const uint4*>(y) + bc * H * (long long)nvec;
-    for (int e = threadIdx.x; e < (kDwVecRows + 2) * nvec; e += blockDim.x) {
-        const int rr = e / nvec, v = e - (e / nvec) * nvec;
-        const int h = h0 - 1 + rr;
-        sband[e] = (h >= 0 && h < H) ? __ldg(yp + (long long)h * nvec + v) : make_uint4(0, 0, 0, 0);
-    }
-    float k[9];
-#pragma unroll
-    for (int m = 0; m < 9; ++m)
-        k[m] = __bfloat162float(__ushort_as_bfloat16(K[c * 9 + m]));
-    __syncthreads();
-    const uint16_t* s16 = reinterpret_cast<const uint16_t*>(sband);
-    uint4* zp = reinterpret_cast<uint4*>(z) + bc * H * (long long)nvec;
-    for (int o = threadIdx.x; o < kDwVecRows * nvec; o += blockDim.x) {
-        const int rr = o / nvec, v = o - (o / nvec) * nvec;
-        const int h = h0 + rr;
-        if (h >= H)
-            continue;
-        // halo rows outside the image were staged as zeros
-        const uint16_t* rows[3] = {s16 + (long long)rr * W + 8 * v,
-                                   s16 + (long long)(rr + 1) * W + 8 * v,
-                                   s16 + (long long)(rr + 2) * W + 8 * v};
-        zp[(long long)h * nvec + v] = dw3x3_row8(rows, v, nvec, k);
+    while (r < r1) {
+        const long long pc = r / H;
+        const int hs = (int)(r - pc * H);
+        const int he = (int)((r1 - r) < (long long)(H - hs) ? hs + (r1 - r) : H);
+        r += he - hs;
+        const long long bc = pc / chunks;
+        const int chunk = (int)(pc - bc * chunks);
+        const int c = (int)(bc % C);
+        const int v = chunk * 32 + lane;
+        const bool act = v < nvec;
+        const uint4* yp = reinterpret_cast<const uint4*>(y) + bc * H * (long long)nvec;
+        const uint16_t* y16 = y + bc * H * (long long)W;
+        uint4* zp = reinterpret_cast<uint4*>(z) + bc * H * (long long)nvec;
+        uint64_t k2[9];
+        dw_weights(K + c * 9, k2);
+        // input rows hs-1 .. he are needed; row x goes to slot (x - hs + 1) % kDwRing
+        auto fetch = [&](int x) {
+            const bool ok = act && x >= 0 && x < H && x <= he;
+            const int slot = (x - hs + 1) % kDwRing;
+            cp_async_16z(ring0 + (uint32_t)(slot * 32 * 16), ok ? yp + (long long)x * nvec + v : yp,
+                         ok ? 16u : 0u);
+            cp_async_commit();
+        };
+        // row x -> pairs (after its copy completed), then its slot is refilled
+        auto take = [&](int x, DwRowPairs& u) {
+            cp_async_wait_group<kDwRing - 1>();
+            const uint4 vec = ringp[((x - hs + 1) % kDwRing) * 32];
+            const bool hv = x >= 0 && x < H && x <= he;
+            uint32_t lf = __shfl_up_sync(0xffffffffu, vec.w, 1) & 0xFFFF0000u;
+            uint32_t rt = __shfl_down_sync(0xffffffffu, vec.x, 1) << 16;
+            if (lane == 0)
+                lf = (act && hv && v > 0) ? (uint32_t)__ldg(y16 + (long long)x * W + 8 * v - 1) << 16
+                                          : 0u;
+            if (lane == 31)
+                rt = (act && hv && v + 1 < nvec)
+                         ? (uint32_t)__ldg(y16 + (long long)x * W + 8 * v + 8) << 16
+                         : 0u;
+            dw_unpack(vec, lf, rt, u);
+            fetch(x + kDwRing);
+        };
+        auto emit = [&](int h, const DwRowPairs& u0, const DwRowPairs& u1, const DwRowPairs& u2) {
+            const DwRowPairs u[3] = {u0, u1, u2};
+            const uint4 out = dw3x3_pairs8(u, k2);
+            if (act)
+                zp[(long long)h * nvec + v] = out;
+        };
+        for (int i = 0; i < kDwRing; ++i)
+            fetch(hs - 1 + i);
+        DwRowPairs ua, ub, uc;
+        take(hs - 1, ua);
+        take(hs, ub);
+        // three rows per pass, the unpacked rows rotating through ua, ub, uc
+        for (int h = hs; h < he; h += 3) {
+            take(h + 1, uc);
+            emit(h, ua, ub, uc);
+            if (h + 1 >= he)
+                break;
+            take(h + 2, ua);
+            emit(h + 1, ub, uc, ua);
+            if (h + 2 >= he)
+                break;
+            take(h + 3, ub);
+            emit(h + 2, uc, ua, ub);
+        }
+        cp_async_wait_group<0>();   // the ring is free before the next segment
     }
 }
 
@@ -599,16 +653,19 @@ cudaError_t dw3x3_launch(const Geom& g, bool is_bf16, const void* y, const void*
 {
     if (is_bf16 && g.W % 8 == 0 && reinterpret_cast<uintptr_t>(y) % 16 == 0 &&
         reinterpret_cast<uintptr_t>(z) % 16 == 0) {
-        const int ty = (g.H + kDwVecRows - 1) / kDwVecRows;
-        const long long blocks = (long long)g.B * g.C * ty;
-        const size_t smem = (size_t)(kDwVecRows + 2) * (g.W / 8) * 16;
-        if (blocks > 0 && blocks <= 0x7fffffffLL && smem <= kSimtSmemMax) {
-            cudaError_t e = set_smem(dw3x3_bf16_vec_kernel, smem);
-            if (e == cudaSuccess)
-                e = launch_pdl(dw3x3_bf16_vec_kernel, dim3((unsigned)blocks), dim3(256), smem,
-                               L.stream, static_cast<const uint16_t*>(y),
-                               static_cast<const uint16_t*>(K), static_cast<uint16_t*>(z), g.C,
-                               g.H, g.W, ty);
+        const int chunks = (g.W / 8 + 31) / 32;
+        const long long total_rows = (long long)g.B * g.C * chunks * g.H;
+        // one pass of warps over the SMs; at least 8 rows per warp
+        long long blocks = (long long)L.num_sms * kDwBlocksPerSm;
+        const long long need = (total_rows + 8 * kDwWarps - 1) / (8 * kDwWarps);
+        if (blocks > need)
+            blocks = need;
+        if (blocks > 0) {
+            cudaError_t e = launch_pdl(dw3x3_bf16_rows_kernel, dim3((unsigned)blocks),
+                                       dim3(kDwWarps * 32), kDwSmem, L.stream,
+                                       static_cast<const uint16_t*>(y),
+                                       static_cast<const uint16_t*>(K), static_cast<uint16_t*>(z),
+                                       g.C, g.H, g.W, chunks, total_rows);
             if (e != cudaSuccess)
                 return e;
             note_launches(1);

@@ -543,10 +543,8 @@ __global__ void __launch_bounds__(kThreads, 1) wbmm_tc_fwd_kernel(const __grid_c
                 const int left = P.bands - ub0;
                 const int planes = (left < P.ub ? left : P.ub) / P.nh;
                 const int b0 = ub0 / P.nh;
-                float kw[9];
-#pragma unroll
-                for (int m = 0; m < 9; ++m)
-                    kw[m] = __bfloat162float(__ushort_as_bfloat16(P.dw[t.c * 9 + m]));
+                uint64_t kw[9];
+                dw_weights(P.dw + t.c * 9, kw);
                 const int nvec = P.W / 8, per_plane = P.H * nvec;
                 for (int o = et; o < planes * per_plane; o += kEpiWarps * 32) {
                     const int j = o / per_plane, r = o - j * per_plane;
