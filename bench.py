@@ -99,6 +99,8 @@ def kernel_bytes(wl, name):
     tbl = wl.C * wl.t * e
     return {"forward": 2 * m + tbl, "backward_dx": 2 * m + tbl,
             "backward_dt": 2 * m + wl.C * wl.t * 4,
+            # x, dY (once), dX, T, dT: both gradients in one call
+            "backward": 3 * m + tbl + wl.C * wl.t * 4,
             "forward_cached": 2 * m + wl.C * wl.d * wl.d * e,
             "forward_cached_dw3x3": 2 * m + wl.C * wl.d * wl.d * e + wl.C * 9 * e,
             "reparam_merge": wl.C * wl.d * wl.d * e + tbl,
@@ -113,6 +115,8 @@ def kernel_flops(wl, name):
         return 2.0 * n * wl.d + 18.0 * n
     if name == "reparam_merge":
         return float(wl.C * wl.d * wl.d)
+    if name == "backward":
+        return 4.0 * n * wl.d
     return 2.0 * n * wl.d
 
 
@@ -211,10 +215,13 @@ class Arm:
                 s["z"] = torch.empty_like(s["x"])
 
     def kernels(self):
-        """The step's kernels, one call each (the per-kernel breakdown)."""
+        """The step's launch units, one call each (the per-call breakdown).
+        The training step's backward call launches the input-gradient and
+        table-gradient kernels side by side on disjoint SMs; it is timed as
+        one unit."""
         k = self.wl.kind
         if k == "train":
-            return ["forward", "backward_dx", "backward_dt"]
+            return ["forward", "backward"]
         if k == "cached_dw":
             return ["forward_cached", "dw3x3"]
         if k == "reparam":
@@ -227,13 +234,14 @@ class Arm:
         where its stencil work blocks the epilogue warps)."""
         if self.wl.kind == "reparam":
             return ["reparam_merge"]    # one-time preparation of the inference matrix
+        if self.wl.kind == "train":
+            # one gradient per call: each kernel alone on the whole device
+            return ["backward_dx", "backward_dt"]
         return ["forward_cached_dw3x3"] if self.wl.kind == "cached_dw" else []
 
     def calls(self):
         """The step as a user issues it: the training step is one forward
         and one backward call that returns both dX and dT."""
-        if self.wl.kind == "train":
-            return ["forward", "backward"]
         return self.kernels()
 
     def launch(self, name, s):
@@ -289,8 +297,13 @@ def prefill(ms=20.0):
 
 def recorded_traffic(kernel):
     """DRAM bytes per launch from the committed ncu capture, or None when the
-    kernel source changed since the counters were taken."""
+    kernel source changed since the counters were taken.  The backward call
+    is the sum of its two kernels' captures (ncu runs them one after the
+    other, so the second read of dY counts again)."""
     import hashlib
+    if kernel == "backward":
+        parts = [recorded_traffic("backward_dx"), recorded_traffic("backward_dt")]
+        return None if None in parts else sum(parts)
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
             rec = json.load(f).get(kernel)
@@ -382,9 +395,6 @@ def run_gpu(args, rank, world, local_rank):
     barrier(world)
     ms_total = max_over_ranks(e0.elapsed_time(e1), world, dev)
     ms_step = ms_total / K
-    # graph replays launch the captured kernels: count them per step
-    per_step_launches = len(wb_arm.kernels())
-    gpu_launches = per_step_launches * K
     assert wb.wbmm_launch_count() == launches0   # graphs: no host launches
 
     # ---- region B: the same steps launched eagerly, events around each kernel
@@ -394,6 +404,7 @@ def run_gpu(args, rank, world, local_rank):
     barrier(world)
     torch.cuda.synchronize()
     prefill()
+    launches1 = wb.wbmm_launch_count()
     for k in range(K):
         s = wb_arm.sets[k % len(wb_arm.sets)]
         for j, name in enumerate(names):
@@ -402,6 +413,8 @@ def run_gpu(args, rank, world, local_rank):
             evs[k][j][1].record(stream)
     torch.cuda.synchronize()
     barrier(world)
+    # the graph replays launch the same kernels as these eager steps
+    gpu_launches = wb.wbmm_launch_count() - launches1
     alt = {}
     for name in wb_arm.alternatives():
         s = wb_arm.sets[0]
@@ -509,6 +522,9 @@ def run_gpu(args, rank, world, local_rank):
                               "frac": round(kern[dom]["gbs"] / peaks["hbm_gbs"], 4),
                               "traffic": recorded_traffic(dom) if wl.name == "train_bf16" else None,
                               "peak_source": peaks["source"]}
+        if dom == "backward":
+            result["roofline"]["launch"] = ("one backward call: the dX and dT kernels side by "
+                                            "side on disjoint SMs; bytes x + dY + dX + T + dT")
     else:
         result["roofline"] = {"bound": "tensor", "kernel": dom, "achieved": kern[dom]["tflops"],
                               "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",

@@ -117,6 +117,29 @@ def test_dt_is_deterministic():
         assert torch.equal(r, runs[0])
 
 
+def test_backward_both_gradients_share_the_device():
+    # enough table-gradient tiles (40 channels x 16) for the two gradient
+    # kernels to run side by side on disjoint SMs: dX equals the dX-only
+    # call bit for bit (windows are independent of the grid), dT is
+    # deterministic and within tolerance of the dT-only call (another grid,
+    # so another fixed summation order)
+    B, C, H, W, w = 64, 40, 56, 56, 14
+    x, dy = gen((B, C, H, W), 30), gen((B, C, H, W), 31)
+    T = gen((C, 729), 32, scale=0.02)
+    dX1, _ = wb.backward(x, T, dy, w, need_dt=False)
+    _, dT1 = wb.backward(x, T, dy, w, need_dx=False)
+    runs = [wb.backward(x, T, dy, w) for _ in range(3)]
+    torch.cuda.synchronize()
+    assert wb.wbmm_get_device_status() == 0
+    for dX, dT in runs:
+        assert torch.equal(dX, dX1)
+        assert torch.equal(dT, runs[0][1])
+    xr, gr = to_np(x[:, :4]), to_np(dy[:, :4])
+    check_bf16(to_np(runs[0][1][:4]), oracle.backward_dt(xr, gr, w), dt_bound(xr, gr, w),
+               "dT with dX")
+    check_bf16(to_np(runs[0][1]), to_np(dT1), dt_bound(to_np(x), to_np(dy), w), "dT vs dT-only")
+
+
 # Degenerate and boundary window sizes: w = 1 (each channel a scalar gain,
 # CUDA-core path), one window per image (tensor-core path, nh = nw = 1),
 # w = 32 (largest register-tiled CUDA-core size) and w = 40 (plain CUDA-core

@@ -94,7 +94,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
         return true;
     const long long t0 = clock64();
     while (true) {
-        if (mbar_try_wait_sleep(bar, parity, 20000))
+        if (mbar_try_wait(bar, parity))
             return true;
         if (*abort)
             return false;

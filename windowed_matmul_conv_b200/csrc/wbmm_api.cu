@@ -251,9 +251,22 @@ wbmm_status wbmm_backward(const void* x, const void* T, const void* dY, void* dX
     if ((st = make_launch(stream, &L)) != WBMM_OK)
         return st;
     const bool tc_dt = dT && dt == WBMM_BF16 && tc_dt_supported(g);
+    // Both gradients on tensor cores and enough tiles to fill the device: the
+    // two kernels run at the same time on disjoint SMs (2/5 for dX, the rest
+    // for dT, the measured balance at w = 14), each walking the channels in
+    // the same order, so the second read of each dY tile is served from L2
+    // and one kernel's ramp and tail overlap the other's steady state.  The
+    // dT kernel's grid (and so its fixed summation order) is a function of
+    // the shape and the SM count only.
+    Launch Lx = L, Lt = L;
+    if (dX && tc_dt && tc_toep_supported(g) && tc_dt_tiles(g) >= 2LL * L.num_sms &&
+        L.num_sms >= 5) {
+        Lx.num_sms = (2 * L.num_sms + 2) / 5;
+        Lt.num_sms = L.num_sms - Lx.num_sms;
+    }
     if (dX) {
         if (dt == WBMM_BF16 && tc_toep_supported(g)) {
-            st = from_cuda(tc_toep_launch(g, kTableFlip, dY, T, dX, L));
+            st = from_cuda(tc_toep_launch(g, kTableFlip, dY, T, dX, Lx));
             t_last_path = 1;
         } else if (dt == WBMM_BF16 && tc_fwd_supported(g, false)) {
             st = from_cuda(tc_fwd_launch(g, kTableFlip, dY, T, dX, nullptr, L));
@@ -271,7 +284,7 @@ wbmm_status wbmm_backward(const void* x, const void* T, const void* dY, void* dX
             // dX, when requested, was the launch just before this one (every
             // library kernel signals its dependents only after its own wait)
             const bool after_dx = dX != nullptr;
-            st = from_cuda(tc_dt_launch(g, x, dY, part, dT, after_dx, L));
+            st = from_cuda(tc_dt_launch(g, x, dY, part, dT, after_dx, Lt));
         } else {
             st = from_cuda(simt_dt_launch(g, dt == WBMM_BF16, x, dY, part, L));
             if (st != WBMM_OK)

@@ -75,9 +75,11 @@ cudaError_t tc_cached_launch(const Geom& g, const void* x, const void* M, void* 
 // tables of channels split between CTAs and one flag word per table.
 // after_dx: the previous launch on the stream is the same backward call's
 // input-gradient kernel (which reads dY and T and writes only dX), so the
-// kernel need not wait for it to finish.
+// kernel need not wait for it to finish.  The grid is min(L.num_sms, 256,
+// tiles); tc_dt_tiles is the number of 64-window (32 at w >= 15) tiles.
 bool tc_dt_supported(const Geom& g);
 long long tc_dt_partials(const Geom& g);
+long long tc_dt_tiles(const Geom& g);
 long long tc_dt_workspace_floats(const Geom& g);
 cudaError_t tc_dt_launch(const Geom& g, const void* x, const void* dy, float* workspace, float* dT,
                          bool after_dx, const Launch& L);

@@ -738,6 +738,11 @@ long long tc_dt_partials(const Geom& g)
     return tc_dt_partials_impl(g);
 }
 
+long long tc_dt_tiles(const Geom& g)
+{
+    return (long long)g.C * dt_tiles_per_channel(g);
+}
+
 long long tc_dt_workspace_floats(const Geom& g)
 {
     // partial tables, then one 64-bit flag per table (8-byte aligned)

@@ -24,14 +24,15 @@
 // of K slots), so shared memory holds only Q, the raw load ring and two
 // output staging buffers, and a tile's input and output never share a buffer.
 //
-// Warp roles (480 threads):
+// Warp roles (608 threads):
 //   warp 0       producer: bulk/TMA copies of half tiles (whole bands) into a
 //                ring of raw slots
 //   warp 1       MMA issuer (one thread) and TMEM owner
 //   warp 2       storer: stores a finished tile from its output buffer
-//   warps 3..6   transform: one per TMEM lane quarter; thread = window, raw
-//                band layout -> A rows in TMEM (two A stages)
-//   warps 7..14  epilogue: TMEM -> bf16 output rows -> band layout in an
+//   warps 3..10  transform: two per TMEM lane quarter, each taking half of
+//                the window rows; thread = window, raw band layout -> A rows
+//                in TMEM (two A stages)
+//   warps 11..18 epilogue: TMEM -> bf16 output rows -> band layout in an
 //                output buffer.  They also write Q: the CTA's first two
 //                channels up front, and Q of channel ci+1 right after the
 //                first tile of channel ci, whose completion implies that
@@ -73,14 +74,27 @@ struct ToepCfg {
     static constexpr int LOADS = (NP + 31) / 32;             // 32-column TMEM loads per row
     static constexpr int RL = 32 / RP;                       // window rows per load
     static constexpr uint32_t IDESC = idesc_bf16(128, NP);
+    // With one 128-window M tile (RP = 16), the accumulator is two halves of
+    // output rows, [0, P0) and [P0, w), at TMEM columns 256 and 384: the MMAs
+    // of one half run while the epilogue drains the other.
+    static constexpr bool NSPLIT = MTW == 1;
+    static constexpr int P0 = (WS + 1) / 2;
+    static constexpr int N0 = NSPLIT ? P0 * RP : NP;
+    static constexpr int N1 = NSPLIT ? WS * RP - N0 : 16;
+    static constexpr uint32_t IDESC0 = idesc_bf16(128, N0);
+    static constexpr uint32_t IDESC1 = idesc_bf16(128, N1);
     static_assert(MTW * A_COLS <= 128, "an A stage fits in 128 TMEM columns");
     static_assert((MTW - 1) * DSTEP + NP <= 256, "the accumulator fits in 256 TMEM columns");
     static_assert((WS - 1) * RP % 8 == 0, "Q row offsets must be whole core matrices");
+    static_assert(!NSPLIT || (RP == 16 && N0 <= 128 && N1 <= 128 && N0 % 16 == 0 &&
+                              N1 % 16 == 0 && N1 >= 16),
+                  "each accumulator half fits in 128 TMEM columns");
 };
 
 constexpr int kToepRing = 8;
 constexpr int kToepXformWarp0 = 3;
-constexpr int kToepEpiWarp0 = kToepXformWarp0 + 4;
+constexpr int kToepXformWarps = 8;
+constexpr int kToepEpiWarp0 = kToepXformWarp0 + kToepXformWarps;
 constexpr int kToepEpiWarps = 8;
 constexpr int kToepThreads = (kToepEpiWarp0 + kToepEpiWarps) * 32;
 
@@ -112,8 +126,8 @@ struct ToepBars {
     uint64_t a_full[2];     // A stage written by the transform
     uint64_t a_empty[2];    // A stage's MMAs have completed
     uint64_t q_full[2];
-    uint64_t acc_full;
-    uint64_t acc_empty;
+    uint64_t acc_full[2];   // per accumulator half (one when not split)
+    uint64_t acc_empty[2];
     uint64_t out_full[2];   // buffer holds the tile's output
     uint64_t out_empty[2];  // buffer has been read by the storer
     uint64_t fin;
@@ -188,15 +202,15 @@ __device__ __forceinline__ void build_q(uint8_t* q, const uint16_t* tst, int tid
     }
 }
 
-// One window's rows -> its TMEM lane of an A stage: window row r at columns
-// r*RP/2 .. (r+1)*RP/2 - 1 (slot pairs), rows w .. RROWS-1 zero.
-template <int WS>
+// Rows [R0, R1) of one window -> its TMEM lane of an A stage: window row r
+// at columns r*RP/2 .. (r+1)*RP/2 - 1 (slot pairs), rows w .. RROWS-1 zero.
+template <int WS, int R0, int R1>
 __device__ __forceinline__ void window_to_tmem(const uint16_t* src0, bool valid, int W,
                                                uint32_t acol)
 {
     using F = ToepCfg<WS>;
 #pragma unroll 2
-    for (int r = 0; r < F::RROWS; ++r) {
+    for (int r = R0; r < R1; ++r) {
         uint32_t wv[F::RP / 2];
         if (valid && r < WS) {
             const uint16_t* src = src0 + r * W;
@@ -254,17 +268,19 @@ __global__ void __launch_bounds__(kToepThreads, 1)
     if (threadIdx.x == 0) {
         for (int i = 0; i < kToepRing; ++i) {
             mbar_init(&S.raw_full[i], 1);
-            mbar_init(&S.raw_empty[i], 4);
+            mbar_init(&S.raw_empty[i], kToepXformWarps);
         }
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&S.a_full[i], 4);
+            mbar_init(&S.a_full[i], kToepXformWarps);
             mbar_init(&S.a_empty[i], 1);
             mbar_init(&S.q_full[i], kToepEpiWarps);
             mbar_init(&S.out_full[i], kToepEpiWarps);
             mbar_init(&S.out_empty[i], 1);
         }
-        mbar_init(&S.acc_full, 1);
-        mbar_init(&S.acc_empty, kToepEpiWarps);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&S.acc_full[i], 1);
+            mbar_init(&S.acc_empty[i], kToepEpiWarps);
+        }
         mbar_init(&S.fin, 1);
         S.abort = 0;
         fence_mbar_init();
@@ -353,16 +369,42 @@ __global__ void __launch_bounds__(kToepThreads, 1)
                 if (first)
                     ok = ok && mbar_wait(&S.q_full[qb], (ci >> 1) & 1, abort, P.budget, P.status);
                 ok = ok && mbar_wait(&S.a_full[st], (seq >> 1) & 1, abort, P.budget, P.status);
-                if (seq >= 1)
-                    ok = ok && mbar_wait(&S.acc_empty, (seq - 1) & 1, abort, P.budget, P.status);
                 if (!ok)
                     continue;
-                tc_fence_after();
                 // K step k: A columns 8k .. 8k+7 of the M tile, Q rows from
                 // (w - 1 - G*k)*RP: only the start-address field moves.
                 const uint64_t qdesc0 = smem_desc(
                     smem_u32(q_base + (size_t)qb * F::Q_BYTES) + (uint32_t)((WS - 1) * F::RP * 32),
                     128, 256);
+                if constexpr (F::NSPLIT) {
+                    const uint32_t a0 = tmem + (uint32_t)(st * 128);
+#pragma unroll
+                    for (int hN = 0; hN < 2; ++hN) {
+                        if (seq >= 1)
+                            ok = ok && mbar_wait(&S.acc_empty[hN], (seq - 1) & 1, abort, P.budget,
+                                                 P.status);
+                        if (!ok)
+                            break;
+                        tc_fence_after();
+                        // half hN: output rows from hN*P0, i.e. Q rows N0*hN on
+                        const uint64_t qd = qdesc0 + (uint64_t)(hN * F::N0 * 2);
+                        const uint32_t d = tmem + 256u + (uint32_t)(hN * 128);
+#pragma unroll
+                        for (int k = 0; k < F::KSTEPS; ++k)
+                            mma_ts(d, a0 + (uint32_t)(k * 8),
+                                   qd - (uint64_t)(k * F::G * F::RP * 2),
+                                   hN ? F::IDESC1 : F::IDESC0, k > 0 ? 1u : 0u);
+                        tc_commit(&S.acc_full[hN]);
+                    }
+                    if (ok)
+                        tc_commit(&S.a_empty[st]);
+                    continue;
+                }
+                if (seq >= 1)
+                    ok = ok && mbar_wait(&S.acc_empty[0], (seq - 1) & 1, abort, P.budget, P.status);
+                if (!ok)
+                    continue;
+                tc_fence_after();
 #pragma unroll
                 for (int mt = 0; mt < F::MTW; ++mt) {
                     const uint32_t a0 = tmem + (uint32_t)(st * 128 + mt * F::A_COLS);
@@ -374,7 +416,7 @@ __global__ void __launch_bounds__(kToepThreads, 1)
                                k > 0 ? 1u : 0u);
                 }
                 tc_commit(&S.a_empty[st]);
-                tc_commit(&S.acc_full);
+                tc_commit(&S.acc_full[0]);
             }
             // Drain: all issued MMAs complete before TMEM is released.
             tc_commit(&S.fin);
@@ -413,10 +455,13 @@ __global__ void __launch_bounds__(kToepThreads, 1)
         bulk_wait<0>();
     } else if (warp < kToepEpiWarp0) {
         // ------------------------------------------------------ transform
-        // Thread = window mt*128 + quarter*32 + lane.  tcgen05.st writes all
-        // 32 lanes of the quarter, so a tile is written once both halves
-        // have landed.
+        // Thread = window mt*128 + quarter*32 + lane; warp part 0 writes the
+        // first half of the window rows, part 1 the rest.  tcgen05.st writes
+        // all 32 lanes of the quarter, so a tile is written once both halves
+        // of the tile have landed.
+        constexpr int RH = (F::RROWS + 1) / 2;
         const int quarter = warp & 3;
+        const int part = (warp - kToepXformWarp0) >> 2;
         const uint32_t lanebase = (uint32_t)(quarter * 32) << 16;
         for (int seq = 0; seq < n_it; ++seq) {
             const BandTile t = toep_tile(P, it0 + seq);
@@ -441,8 +486,11 @@ __global__ void __launch_bounds__(kToepThreads, 1)
                     const uint16_t* raw = reinterpret_cast<const uint16_t*>(
                         raw_base + (size_t)(h ? s1 : s0) * P.sub_bytes);
                     const uint16_t* src0 = raw + (valid ? woff[h ? n - h0win : n] : 0);
-                    window_to_tmem<WS>(src0, valid, P.W,
-                                       tmem + lanebase + (uint32_t)(st * 128 + mt * F::A_COLS));
+                    const uint32_t acol = tmem + lanebase + (uint32_t)(st * 128 + mt * F::A_COLS);
+                    if (part == 0)
+                        window_to_tmem<WS, 0, RH>(src0, valid, P.W, acol);
+                    else
+                        window_to_tmem<WS, RH, F::RROWS>(src0, valid, P.W, acol);
                 }
                 tmem_wait_st();
             }
@@ -485,24 +533,23 @@ __global__ void __launch_bounds__(kToepThreads, 1)
             const int nwin = t.nb * P.nw;
             const int ob = seq % NO;
             bool ok = !*abort;
-            ok = ok && mbar_wait(&S.acc_full, seq & 1, abort, P.budget, P.status);
             if (seq >= NO)
                 ok = ok && mbar_wait(&S.out_empty[ob], ((seq / NO) - 1) & 1, abort, P.budget,
                                      P.status);
-            ok = __all_sync(0xffffffffu, ok);
-            tc_fence_after();
             uint16_t* obuf = reinterpret_cast<uint16_t*>(out_base + (size_t)ob * F::OUT_BYTES);
-#pragma unroll 1
-            for (int mt = 0; mt < F::MTW; ++mt) {
+            // Rows [pb, pe) of every window of M tile mt from the accumulator
+            // columns at lbase (row pb at column 0), warp half hf taking every
+            // other 32-column load; returns after the last TMEM read.
+            auto drain = [&](int mt, uint32_t lbase, int pb, int pe) {
                 const int n = mt * 128 + quarter * 32 + lane;
                 if (!ok || mt * 128 + quarter * 32 >= nwin)
-                    continue;
+                    return;
                 const bool valid = n < nwin;
                 uint16_t* o0 = obuf + (valid ? woff[n] : 0);
-                const uint32_t lrow = tmem + ((uint32_t)(quarter * 32) << 16) + 256u +
-                                      (uint32_t)(mt * F::DSTEP);
+                const uint32_t lrow = tmem + ((uint32_t)(quarter * 32) << 16) + lbase;
+                const int nload = ((pe - pb) * F::RP + 31) / 32;
 #pragma unroll 1
-                for (int li = hf; li < F::LOADS; li += 2) {
+                for (int li = hf; li < nload; li += 2) {
                     uint32_t r[32];
                     tmem_ld32(lrow + (uint32_t)(li * 32), r);
                     tmem_wait_ld(r);
@@ -510,8 +557,8 @@ __global__ void __launch_bounds__(kToepThreads, 1)
                         continue;
 #pragma unroll
                     for (int rr = 0; rr < F::RL; ++rr) {
-                        const int pr = li * F::RL + rr;
-                        if (pr >= WS)
+                        const int pr = pb + li * F::RL + rr;
+                        if (pr >= pe)
                             continue;
                         uint16_t* o = o0 + pr * P.W;
                         if (WS % 2 == 0) {
@@ -527,12 +574,33 @@ __global__ void __launch_bounds__(kToepThreads, 1)
                         }
                     }
                 }
+            };
+            if constexpr (F::NSPLIT) {
+#pragma unroll 1
+                for (int hN = 0; hN < 2; ++hN) {
+                    ok = ok && mbar_wait(&S.acc_full[hN], seq & 1, abort, P.budget, P.status);
+                    ok = __all_sync(0xffffffffu, ok);
+                    tc_fence_after();
+                    drain(0, 256u + (uint32_t)(hN * 128), hN ? F::P0 : 0, hN ? WS : F::P0);
+                    tc_fence_before();
+                    __syncwarp();
+                    if (ok && lane == 0)
+                        mbar_arrive(&S.acc_empty[hN]);
+                }
+            } else {
+                ok = ok && mbar_wait(&S.acc_full[0], seq & 1, abort, P.budget, P.status);
+                ok = __all_sync(0xffffffffu, ok);
+                tc_fence_after();
+#pragma unroll 1
+                for (int mt = 0; mt < F::MTW; ++mt)
+                    drain(mt, 256u + (uint32_t)(mt * F::DSTEP), 0, WS);
             }
             tc_fence_before();
             fence_proxy_async_smem();
             __syncwarp();
             if (ok && lane == 0) {
-                mbar_arrive(&S.acc_empty);
+                if constexpr (!F::NSPLIT)
+                    mbar_arrive(&S.acc_empty[0]);
                 mbar_arrive(&S.out_full[ob]);
             }
             if (t.c != cur_c) {
