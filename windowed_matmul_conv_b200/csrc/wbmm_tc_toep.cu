@@ -304,6 +304,10 @@ __global__ void __launch_bounds__(kToepThreads, 1)
 
     if (warp == 0) {
         // ------------------------------------------------------ producer
+        // The first two tables' loads are issued before any tile's, so that
+        // they are not queued behind every CTA's ring fill (the first MMA
+        // needs Q).
+        named_bar_sync(5, 32 + kToepEpiWarps * 32);
         int issued = 0;
         bool go = true;
         for (int seq = 0; seq < n_it && go; ++seq) {
@@ -511,12 +515,37 @@ __global__ void __launch_bounds__(kToepThreads, 1)
         const int et = threadIdx.x - kToepEpiWarp0 * 32;
         const int c_first = toep_tile(P, it0).c;
         const int nch = toep_tile(P, it0 + n_it - 1).c - c_first + 1;
+        // The tables of the CTA's first two channels, loaded into registers
+        // before the producer may start: the rest of the tables are read
+        // while Q of the channel before is in use.
+        constexpr int TPT = (F::TSZ + kToepEpiWarps * 32 - 1) / (kToepEpiWarps * 32);
+        uint16_t tpre[2][TPT];
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+            for (int i = 0; i < TPT; ++i) {
+                const int e = et + i * kToepEpiWarps * 32;
+                tpre[j][i] = (j < nch && e < F::TSZ)
+                                 ? __ldg(reinterpret_cast<const unsigned short*>(P.T) +
+                                         (long long)(c_first + j) * F::TSZ + e)
+                                 : (uint16_t)0;
+            }
+        named_bar_arrive(5, 32 + kToepEpiWarps * 32);
         // Every epilogue warp takes part in every build, whatever its wait
         // results, so the named barriers always see all 256 threads.
         auto build_for = [&](int ci) {
             named_bar_sync(2, kToepEpiWarps * 32);     // staged table fully read
-            stage_table<WS, MODE>(tst, P.T + (long long)(c_first + ci) * F::TSZ, et,
-                                  kToepEpiWarps * 32);
+            if (ci < 2) {
+#pragma unroll
+                for (int i = 0; i < TPT; ++i) {
+                    const int e = et + i * kToepEpiWarps * 32;
+                    if (e < F::TSZ)
+                        tst[MODE == kTable ? e : F::TSZ - 1 - e] = tpre[ci][i];
+                }
+            } else {
+                stage_table<WS, MODE>(tst, P.T + (long long)(c_first + ci) * F::TSZ, et,
+                                      kToepEpiWarps * 32);
+            }
             named_bar_sync(2, kToepEpiWarps * 32);
             build_q<WS>(q_base + (size_t)(ci & 1) * F::Q_BYTES, tst, et, kToepEpiWarps * 32);
             fence_proxy_async_smem();
