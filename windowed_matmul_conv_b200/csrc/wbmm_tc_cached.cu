@@ -14,23 +14,27 @@
 // warps with tcgen05.st, which leaves shared memory for the load ring and an
 // output staging buffer.
 //
-// Warp roles (480 threads):
+// Warp roles (608 threads):
 //   warp 0       producer: bulk/TMA copies of half tiles into a ring of raw slots
 //   warp 1       MMA issuer (one thread) and TMEM owner
 //   warp 2       storer: stores a tile from the output staging buffer
-//   warps 3..6   transform: one per TMEM lane quarter; thread = window, raw
-//                band layout -> A rows in TMEM (two A stages)
-//   warps 7..14  epilogue: TMEM -> bf16 output rows -> band layout in the
+//   warps 3..10  transform: two per TMEM lane quarter, each half of the window
+//                rows; thread = window, raw band layout -> A rows in TMEM (two
+//                A stages)
+//   warps 11..18 epilogue: TMEM -> bf16 output rows -> band layout in the
 //                staging buffer; they also build B (M_c^T in the operand
 //                layout) from HBM for the first channel and after the last
 //                tile of each channel, whose completion implies that every
 //                MMA reading the previous B has finished
 //
-// TMEM: A stages at columns 0 and 128, the accumulator (single) at 256.
+// TMEM: A stages at columns 0 and 128; the accumulator at 256, in two halves
+// of output positions (256 and 384) when there are more than 128 of them.
 // Every wait is bounded; a wait that runs out raises the CTA's abort flag and
 // the device status word, and every role then runs its loop without doing
 // work so that all threads reach the drain and the TMEM release.
 #include <cuda_bf16.h>
+
+#include <type_traits>
 
 #include "ptx_sm100.cuh"
 #include "tc_common.cuh"
@@ -56,11 +60,22 @@ struct CachedCfg {
     static constexpr uint32_t OUT_BYTES = (uint32_t)((128 * D * 2 + 127) / 128 * 128);
     static constexpr uint32_t IDESC = idesc_bf16(128, NP);
     static_assert(A_COLS <= 128 && NP <= 256, "TMEM plan: A stages at 0/128, D at 256");
+    // With more than 128 output positions the accumulator is two halves of
+    // positions, [0, N0) at TMEM column 256 and [N0, NP) at 384: the MMAs of
+    // one half run while the epilogue drains the other.
+    static constexpr bool NSPLIT = NP > 128;
+    static constexpr int N0 = NSPLIT ? (NP / 2 + 15) / 16 * 16 : NP;
+    static constexpr int N1 = NSPLIT ? NP - N0 : 16;
+    static constexpr uint32_t IDESC0 = idesc_bf16(128, N0);
+    static constexpr uint32_t IDESC1 = idesc_bf16(128, N1);
+    static_assert(!NSPLIT || (N0 <= 128 && N1 <= 128 && N1 >= 16 && N0 % 16 == 0),
+                  "each accumulator half fits in 128 TMEM columns");
 };
 
 constexpr int kCRing = 8;
 constexpr int kCXformWarp0 = 3;
-constexpr int kCEpiWarp0 = kCXformWarp0 + 4;
+constexpr int kCXformWarps = 8;
+constexpr int kCEpiWarp0 = kCXformWarp0 + kCXformWarps;
 constexpr int kCEpiWarps = 8;
 constexpr int kCThreads = (kCEpiWarp0 + kCEpiWarps) * 32;
 constexpr int kCTileWindows = 128;
@@ -86,8 +101,8 @@ struct CachedBars {
     uint64_t a_full[2];
     uint64_t a_empty[2];
     uint64_t b_full;
-    uint64_t acc_full;
-    uint64_t acc_empty;
+    uint64_t acc_full[2];   // per accumulator half (one when not split)
+    uint64_t acc_empty[2];
     uint64_t out_full;
     uint64_t out_empty;
     uint64_t fin;
@@ -206,15 +221,17 @@ __global__ void __launch_bounds__(kCThreads, 1)
     if (threadIdx.x == 0) {
         for (int i = 0; i < kCRing; ++i) {
             mbar_init(&S.raw_full[i], 1);
-            mbar_init(&S.raw_empty[i], 4);
+            mbar_init(&S.raw_empty[i], kCXformWarps);
         }
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&S.a_full[i], 4);
+            mbar_init(&S.a_full[i], kCXformWarps);
             mbar_init(&S.a_empty[i], 1);
         }
         mbar_init(&S.b_full, kCEpiWarps);
-        mbar_init(&S.acc_full, 1);
-        mbar_init(&S.acc_empty, kCEpiWarps);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&S.acc_full[i], 1);
+            mbar_init(&S.acc_empty[i], kCEpiWarps);
+        }
         mbar_init(&S.out_full, kCEpiWarps);
         mbar_init(&S.out_empty, 1);
         mbar_init(&S.fin, 1);
@@ -302,21 +319,45 @@ __global__ void __launch_bounds__(kCThreads, 1)
                 if (first)
                     ok = ok && mbar_wait(&S.b_full, ci & 1, abort, P.budget, P.status);
                 ok = ok && mbar_wait(&S.a_full[st], (seq >> 1) & 1, abort, P.budget, P.status);
-                if (seq >= 1)
-                    ok = ok && mbar_wait(&S.acc_empty, (seq - 1) & 1, abort, P.budget, P.status);
                 if (!ok)
                     continue;
-                tc_fence_after();
                 // K step k: A columns 8k .. 8k+7 of stage st, B core matrices 2k, 2k+1
                 const uint64_t bdesc0 = smem_desc(smem_u32(b_base), F::LBO_B, F::SBO_B);
                 const uint32_t a0 = tmem + (uint32_t)(st * 128);
+                if constexpr (F::NSPLIT) {
+#pragma unroll
+                    for (int hN = 0; hN < 2; ++hN) {
+                        if (seq >= 1)
+                            ok = ok && mbar_wait(&S.acc_empty[hN], (seq - 1) & 1, abort, P.budget,
+                                                 P.status);
+                        if (!ok)
+                            break;
+                        tc_fence_after();
+                        // half hN: B rows (output positions) from hN*N0, 8-row groups SBO_B apart
+                        const uint64_t bd = bdesc0 + (uint64_t)(hN * (F::N0 / 8) * F::SBO_B / 16);
+#pragma unroll
+                        for (int k = 0; k < F::KSTEPS; ++k)
+                            mma_ts(tmem + 256u + (uint32_t)(hN * 128), a0 + (uint32_t)(k * 8),
+                                   bd + (uint64_t)(k * 2 * F::LBO_B / 16),
+                                   hN ? F::IDESC1 : F::IDESC0, k > 0 ? 1u : 0u);
+                        tc_commit(&S.acc_full[hN]);
+                    }
+                    if (ok)
+                        tc_commit(&S.a_empty[st]);
+                    continue;
+                }
+                if (seq >= 1)
+                    ok = ok && mbar_wait(&S.acc_empty[0], (seq - 1) & 1, abort, P.budget, P.status);
+                if (!ok)
+                    continue;
+                tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < F::KSTEPS; ++k)
                     mma_ts(tmem + 256u, a0 + (uint32_t)(k * 8),
                            bdesc0 + (uint64_t)(k * 2 * F::LBO_B / 16),
                            F::IDESC, k > 0 ? 1u : 0u);
                 tc_commit(&S.a_empty[st]);
-                tc_commit(&S.acc_full);
+                tc_commit(&S.acc_full[0]);
             }
             tc_commit(&S.fin);
             mbar_wait_drain(&S.fin, 0, P.budget, P.status);
@@ -351,9 +392,14 @@ __global__ void __launch_bounds__(kCThreads, 1)
         bulk_wait<0>();
     } else if (warp < kCEpiWarp0) {
         // ------------------------------------------------------ transform
-        // Thread = window n of the warp's lane quarter.  tcgen05.st writes
-        // all 32 lanes, so a tile is written once both halves have landed.
+        // Thread = window n of the warp's lane quarter; warp part 0 writes
+        // the first half of the window rows, part 1 the rest.  tcgen05.st
+        // writes all 32 lanes, so a tile is written once both halves of the
+        // tile have landed.
+        constexpr int RH = (F::RROWS + 1) / 2;
         const int quarter = warp & 3;
+        const int part = (warp - kCXformWarp0) >> 2;
+        const int r_lo = part ? RH : 0, r_hi = part ? F::RROWS : RH;
         const int n = quarter * 32 + lane;
         const uint32_t lanebase = (uint32_t)(quarter * 32) << 16;
         for (int seq = 0; seq < n_it; ++seq) {
@@ -378,7 +424,7 @@ __global__ void __launch_bounds__(kCThreads, 1)
                 const uint16_t* src0 = raw + (valid ? woff[h ? n - h0win : n] : 0);
                 const uint32_t acol = tmem + lanebase + (uint32_t)(st * 128);
 #pragma unroll 2
-                for (int r = 0; r < F::RROWS; ++r) {
+                for (int r = r_lo; r < r_hi; ++r) {
                     uint32_t wv[F::RP / 2];
                     if (valid && r < WS) {
                         const uint16_t* src = src0 + r * P.W;
@@ -437,18 +483,22 @@ __global__ void __launch_bounds__(kCThreads, 1)
             const BandTile t = cached_tile(P, it0 + seq);
             const int nwin = t.nb * P.nw;
             bool ok = !*abort;
-            ok = ok && mbar_wait(&S.acc_full, seq & 1, abort, P.budget, P.status);
             if (seq >= 1)
                 ok = ok && mbar_wait(&S.out_empty, (seq - 1) & 1, abort, P.budget, P.status);
-            ok = __all_sync(0xffffffffu, ok);
-            tc_fence_after();
-            if (ok && quarter * 32 < nwin) {
-                const bool valid = n < nwin;
-                uint16_t* o0 = reinterpret_cast<uint16_t*>(out_base) + (valid ? woff[n] : 0);
-                const uint32_t lrow = tmem + ((uint32_t)(quarter * 32) << 16) + 256u;
-                // accumulator column n is output position (n / w, n % w)
+            const bool valid = n < nwin;
+            uint16_t* o0 = reinterpret_cast<uint16_t*>(out_base) + (valid ? woff[n] : 0);
+            // output positions [E0, E1) from the accumulator columns at lbase
+            // (position E0 at column 0); warp half hf takes every other
+            // 32-column load.  Positions are compile-time constants, so the
+            // (row, column) of each is too.
+            auto drain = [&](uint32_t lbase, auto e0c, auto e1c) {
+                constexpr int E0 = decltype(e0c)::value, E1 = decltype(e1c)::value;
+                if (!ok || quarter * 32 >= nwin)
+                    return;
+                const uint32_t lrow = tmem + ((uint32_t)(quarter * 32) << 16) + lbase;
+                constexpr int NLOAD = (E1 - E0 + 31) / 32;
 #pragma unroll
-                for (int li = 0; li < F::LOADS; ++li) {
+                for (int li = 0; li < NLOAD; ++li) {
                     if ((li & 1) != hf)
                         continue;
                     uint32_t r[32];
@@ -456,30 +506,55 @@ __global__ void __launch_bounds__(kCThreads, 1)
                     tmem_wait_ld(r);
                     if (!valid)
                         continue;
+                    // accumulator column c is output position e0 + c = (e / w, e % w)
                     if (WS % 2 == 0) {
 #pragma unroll
                         for (int j = 0; j < 32; j += 2) {
-                            const int e = li * 32 + j;
-                            if (e < F::D)
+                            const int e = E0 + li * 32 + j;
+                            if (e < E1 && e < F::D)
                                 *reinterpret_cast<uint32_t*>(o0 + (e / WS) * P.W + e % WS) =
                                     cbf16x2_rn(r[j], r[j + 1]);
                         }
                     } else {
 #pragma unroll
                         for (int j = 0; j < 32; ++j) {
-                            const int e = li * 32 + j;
-                            if (e < F::D)
+                            const int e = E0 + li * 32 + j;
+                            if (e < E1 && e < F::D)
                                 o0[(e / WS) * P.W + e % WS] =
                                     __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(r[j])));
                         }
                     }
                 }
+            };
+            if constexpr (F::NSPLIT) {
+#pragma unroll
+                for (int hN = 0; hN < 2; ++hN) {
+                    ok = ok && mbar_wait(&S.acc_full[hN], seq & 1, abort, P.budget, P.status);
+                    ok = __all_sync(0xffffffffu, ok);
+                    tc_fence_after();
+                    if (hN == 0)
+                        drain(256u, std::integral_constant<int, 0>{},
+                              std::integral_constant<int, F::N0>{});
+                    else
+                        drain(384u, std::integral_constant<int, F::N0>{},
+                              std::integral_constant<int, F::NP>{});
+                    tc_fence_before();
+                    __syncwarp();
+                    if (ok && lane == 0)
+                        mbar_arrive(&S.acc_empty[hN]);
+                }
+            } else {
+                ok = ok && mbar_wait(&S.acc_full[0], seq & 1, abort, P.budget, P.status);
+                ok = __all_sync(0xffffffffu, ok);
+                tc_fence_after();
+                drain(256u, std::integral_constant<int, 0>{}, std::integral_constant<int, F::NP>{});
             }
             tc_fence_before();
             fence_proxy_async_smem();
             __syncwarp();
             if (ok && lane == 0) {
-                mbar_arrive(&S.acc_empty);
+                if constexpr (!F::NSPLIT)
+                    mbar_arrive(&S.acc_empty[0]);
                 mbar_arrive(&S.out_full);
             }
             // the channel's last tile is done: every MMA that read B has
