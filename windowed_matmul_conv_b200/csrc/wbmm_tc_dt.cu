@@ -106,8 +106,10 @@ struct TcDtParams {
     int tpc;                // tiles per channel
     int bands;
     int rq, rr;             // range split: CTA k gets rq + (k < rr) tiles
-    int dep_wait;           // 0: the previous kernel reads only what this one
-                            // reads and writes nothing it touches
+    int dep_wait;           // 1: wait for the previous kernel before any load;
+                            // 0: the previous kernel is the same call's input
+                            // gradient, which writes nothing this one touches,
+                            // so the wait moves to the end of the kernel
     int use_tmap;           // tiles are whole planes: one 4-D TMA per tensor
     int kimg;               // planes per tile when use_tmap
     int R;                  // raw ring depth (tiles)
@@ -574,6 +576,12 @@ __global__ void __launch_bounds__(kDtThreads, 1) wbmm_tc_dt_kernel(const __grid_
         __syncwarp();
         tmem_dealloc(tmem, 512);
     }
+    // Without the wait at the start, this grid could finish before the
+    // input-gradient kernel launched ahead of it; a later kernel in the
+    // stream that waits only for this grid would then see dX incomplete.
+    // Waiting here makes this grid's completion imply the earlier one's.
+    if (!P.dep_wait)
+        grid_dep_wait();
 }
 
 // ------------------------------------------------------------------ host
