@@ -94,6 +94,50 @@ __device__ __forceinline__ uint4 dw3x3_pairs8(const DwRowPairs (&u)[3], const ui
     return make_uint4(packed[0], packed[1], packed[2], packed[3]);
 }
 
+// The same ten input values of one row as plain fp32 (v[0] = left
+// neighbour, v[1..8] = the vector, v[9] = right neighbour).
+struct DwRowF {
+    float v[10];
+};
+
+__device__ __forceinline__ void dw_unpack_f(const uint4& vec, uint32_t lf, uint32_t rt, DwRowF& u)
+{
+    const uint32_t w4[4] = {vec.x, vec.y, vec.z, vec.w};
+    u.v[0] = __uint_as_float(lf);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        u.v[1 + 2 * j] = __uint_as_float(w4[j] << 16);
+        u.v[2 + 2 * j] = __uint_as_float(w4[j] & 0xFFFF0000u);
+    }
+    u.v[9] = __uint_as_float(rt);
+}
+
+// dw3x3_pairs8 with one fp32 fused multiply-add per instruction: the same
+// operations on every output in the same order, so the same bits.
+__device__ __forceinline__ uint4 dw3x3_f8(const DwRowF& u0, const DwRowF& u1, const DwRowF& u2,
+                                          const float (&k)[9])
+{
+    float acc[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+        acc[j] = 0.0f;
+    const DwRowF* rows[3] = {&u0, &u1, &u2};
+#pragma unroll
+    for (int a = 0; a < 3; ++a)
+#pragma unroll
+        for (int e = 0; e < 3; ++e)
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                acc[j] = __fmaf_rn(k[a * 3 + e], rows[a]->v[j + e], acc[j]);
+    uint32_t packed[4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        const __nv_bfloat162 v = __floats2bfloat162_rn(acc[2 * m], acc[2 * m + 1]);
+        packed[m] = *reinterpret_cast<const uint32_t*>(&v);
+    }
+    return make_uint4(packed[0], packed[1], packed[2], packed[3]);
+}
+
 // rows[a] points at element 8*v of input row h-1+a, or is null for a row
 // outside the image (read as zeros); v is the vector index in the row and
 // nvec the vectors per row (W / 8).

@@ -327,11 +327,13 @@ __global__ void dw3x3_kernel(const TIn* __restrict__ y, const TIn* __restrict__ 
 // back once, unpacked into fp32 pairs (its left and right neighbour values
 // from the adjacent lanes by shuffles, or a 2-byte load at a chunk edge inside
 // the row), and its slot is refilled at once.  The three live rows stay
-// unpacked in registers.  The per-output arithmetic is dw3x3_pairs8, as in
-// every other bf16 3x3 path, so all of them give the same bits.
+// unpacked in registers.  The per-output arithmetic is dw3x3_f8: the fp32
+// fused multiply-adds of dw3x3_pairs8 (the fused epilogue's, two outputs per
+// instruction) one output at a time in the same order, so both give the same
+// bits.
 constexpr int kDwRing = 16;
 constexpr int kDwWarps = 4;
-constexpr int kDwBlocksPerSm = 4;
+constexpr int kDwBlocksPerSm = 6;
 constexpr size_t kDwSmem = (size_t)kDwWarps * kDwRing * 32 * 16;
 
 __global__ void __launch_bounds__(kDwWarps * 32, kDwBlocksPerSm) dw3x3_bf16_rows_kernel(
@@ -363,8 +365,10 @@ __global__ void __launch_bounds__(kDwWarps * 32, kDwBlocksPerSm) dw3x3_bf16_rows
         const uint4* yp = reinterpret_cast<const uint4*>(y) + bc * H * (long long)nvec;
         const uint16_t* y16 = y + bc * H * (long long)W;
         uint4* zp = reinterpret_cast<uint4*>(z) + bc * H * (long long)nvec;
-        uint64_t k2[9];
-        dw_weights(K + c * 9, k2);
+        float k[9];
+#pragma unroll
+        for (int m = 0; m < 9; ++m)
+            k[m] = __bfloat162float(__ushort_as_bfloat16(__ldg(K + c * 9 + m)));
         // input rows hs-1 .. he are needed; row x goes to slot (x - hs + 1) % kDwRing
         auto fetch = [&](int x) {
             const bool ok = act && x >= 0 && x < H && x <= he;
@@ -374,7 +378,7 @@ __global__ void __launch_bounds__(kDwWarps * 32, kDwBlocksPerSm) dw3x3_bf16_rows
             cp_async_commit();
         };
         // row x -> pairs (after its copy completed), then its slot is refilled
-        auto take = [&](int x, DwRowPairs& u) {
+        auto take = [&](int x, DwRowF& u) {
             cp_async_wait_group<kDwRing - 1>();
             const uint4 vec = ringp[((x - hs + 1) % kDwRing) * 32];
             const bool hv = x >= 0 && x < H && x <= he;
@@ -387,18 +391,17 @@ __global__ void __launch_bounds__(kDwWarps * 32, kDwBlocksPerSm) dw3x3_bf16_rows
                 rt = (act && hv && v + 1 < nvec)
                          ? (uint32_t)__ldg(y16 + (long long)x * W + 8 * v + 8) << 16
                          : 0u;
-            dw_unpack(vec, lf, rt, u);
+            dw_unpack_f(vec, lf, rt, u);
             fetch(x + kDwRing);
         };
-        auto emit = [&](int h, const DwRowPairs& u0, const DwRowPairs& u1, const DwRowPairs& u2) {
-            const DwRowPairs u[3] = {u0, u1, u2};
-            const uint4 out = dw3x3_pairs8(u, k2);
+        auto emit = [&](int h, const DwRowF& u0, const DwRowF& u1, const DwRowF& u2) {
+            const uint4 out = dw3x3_f8(u0, u1, u2, k);
             if (act)
                 zp[(long long)h * nvec + v] = out;
         };
         for (int i = 0; i < kDwRing; ++i)
             fetch(hs - 1 + i);
-        DwRowPairs ua, ub, uc;
+        DwRowF ua, ub, uc;
         take(hs - 1, ua);
         take(hs, ub);
         // three rows per pass, the unpacked rows rotating through ua, ub, uc
