@@ -335,6 +335,7 @@ constexpr int kDwRing = 16;
 constexpr int kDwWarps = 4;
 constexpr int kDwBlocksPerSm = 6;
 constexpr size_t kDwSmem = (size_t)kDwWarps * kDwRing * 32 * 16;
+static_assert((kDwRing & (kDwRing - 1)) == 0, "ring slots advance by masking");
 
 __global__ void __launch_bounds__(kDwWarps * 32, kDwBlocksPerSm) dw3x3_bf16_rows_kernel(
     const uint16_t* __restrict__ y, const uint16_t* __restrict__ K, uint16_t* __restrict__ z,
@@ -369,53 +370,70 @@ __global__ void __launch_bounds__(kDwWarps * 32, kDwBlocksPerSm) dw3x3_bf16_rows
 #pragma unroll
         for (int m = 0; m < 9; ++m)
             k[m] = __bfloat162float(__ushort_as_bfloat16(__ldg(K + c * 9 + m)));
-        // input rows hs-1 .. he are needed; row x goes to slot (x - hs + 1) % kDwRing
-        auto fetch = [&](int x) {
-            const bool ok = act && x >= 0 && x < H && x <= he;
-            const int slot = (x - hs + 1) % kDwRing;
-            cp_async_16z(ring0 + (uint32_t)(slot * 32 * 16), ok ? yp + (long long)x * nvec + v : yp,
-                         ok ? 16u : 0u);
+        // Input rows hs-1 .. he are needed; those inside the image are
+        // [xlo, xhi].  Row x goes to ring slot (x - hs + 1) mod kDwRing; the
+        // fetch and take positions advance one row at a time.
+        const int xlo = hs - 1 > 0 ? hs - 1 : 0, xhi = he < H - 1 ? he : H - 1;
+        int fx = hs - 1;                                    // next row to fetch
+        uint32_t fslot = 0;
+        const uint4* fsrc = yp + (long long)(hs - 1) * nvec + v;
+        auto fetch = [&]() {
+            const bool ok = act && fx >= xlo && fx <= xhi;
+            cp_async_16z(ring0 + fslot * (32u * 16u), ok ? fsrc : yp, ok ? 16u : 0u);
             cp_async_commit();
+            ++fx;
+            fslot = (fslot + 1) & (kDwRing - 1);
+            fsrc += nvec;
         };
-        // row x -> pairs (after its copy completed), then its slot is refilled
-        auto take = [&](int x, DwRowF& u) {
+        int tx = hs - 1;                                    // next row to take
+        uint32_t tslot = 0;
+        const bool edges = chunks > 1;      // a row's chunks need 2-byte edge loads
+        // row tx -> fp32 values (after its copy completed), then its slot is refilled
+        auto take = [&](DwRowF& u) {
             cp_async_wait_group<kDwRing - 1>();
-            const uint4 vec = ringp[((x - hs + 1) % kDwRing) * 32];
-            const bool hv = x >= 0 && x < H && x <= he;
+            const uint4 vec = ringp[tslot * 32];
             uint32_t lf = __shfl_up_sync(0xffffffffu, vec.w, 1) & 0xFFFF0000u;
             uint32_t rt = __shfl_down_sync(0xffffffffu, vec.x, 1) << 16;
             if (lane == 0)
-                lf = (act && hv && v > 0) ? (uint32_t)__ldg(y16 + (long long)x * W + 8 * v - 1) << 16
-                                          : 0u;
-            if (lane == 31)
-                rt = (act && hv && v + 1 < nvec)
-                         ? (uint32_t)__ldg(y16 + (long long)x * W + 8 * v + 8) << 16
-                         : 0u;
+                lf = 0u;
+            if (v + 1 >= nvec)
+                rt = 0u;
+            if (edges) {
+                const bool hv = tx >= xlo && tx <= xhi;
+                if (lane == 0 && act && hv && v > 0)
+                    lf = (uint32_t)__ldg(y16 + (long long)tx * W + 8 * v - 1) << 16;
+                if (lane == 31 && act && hv && v + 1 < nvec)
+                    rt = (uint32_t)__ldg(y16 + (long long)tx * W + 8 * v + 8) << 16;
+            }
             dw_unpack_f(vec, lf, rt, u);
-            fetch(x + kDwRing);
+            ++tx;
+            tslot = (tslot + 1) & (kDwRing - 1);
+            fetch();
         };
-        auto emit = [&](int h, const DwRowF& u0, const DwRowF& u1, const DwRowF& u2) {
+        uint4* zrow = zp + (long long)hs * nvec + v;
+        auto emit = [&](const DwRowF& u0, const DwRowF& u1, const DwRowF& u2) {
             const uint4 out = dw3x3_f8(u0, u1, u2, k);
             if (act)
-                zp[(long long)h * nvec + v] = out;
+                *zrow = out;
+            zrow += nvec;
         };
         for (int i = 0; i < kDwRing; ++i)
-            fetch(hs - 1 + i);
+            fetch();
         DwRowF ua, ub, uc;
-        take(hs - 1, ua);
-        take(hs, ub);
+        take(ua);
+        take(ub);
         // three rows per pass, the unpacked rows rotating through ua, ub, uc
         for (int h = hs; h < he; h += 3) {
-            take(h + 1, uc);
-            emit(h, ua, ub, uc);
+            take(uc);
+            emit(ua, ub, uc);
             if (h + 1 >= he)
                 break;
-            take(h + 2, ua);
-            emit(h + 1, ub, uc, ua);
+            take(ua);
+            emit(ub, uc, ua);
             if (h + 2 >= he)
                 break;
-            take(h + 3, ub);
-            emit(h + 2, uc, ua, ub);
+            take(ub);
+            emit(uc, ua, ub);
         }
         cp_async_wait_group<0>();   // the ring is free before the next segment
     }
