@@ -158,14 +158,21 @@ __device__ __forceinline__ void build_b_global(uint8_t* b, const uint16_t* Mc, i
 {
     using F = CachedCfg<WS>;
     if constexpr (WS % 2 == 0) {
+        // Thread = one 32-bit pair column e of M_c and every RSTEP-th row u
+        // from its phase: the destination column and the row step are fixed,
+        // so each copy costs a few additions.
         constexpr int HALF = F::D / 2;   // 32-bit pairs per row of M_c
-        const uint32_t b32 = smem_u32(b);
-        for (int j = tid; j < F::D * HALF; j += nthreads) {
-            const int u = j / HALF, e = 2 * (j - (j / HALF) * HALF);
+        const int rstep = nthreads / HALF;
+        if (tid < rstep * HALF) {
+            const int ep = tid % HALF, u0 = tid / HALF;
+            const int e = 2 * ep;
             const int k = (e / WS) * F::RP + e % WS;
-            const uint32_t dst = (uint32_t)(u >> 3) * F::SBO_B + (uint32_t)(k >> 3) * F::LBO_B +
-                                 (uint32_t)(u & 7) * 16 + (uint32_t)(k & 7) * 2;
-            cp_async_4(b32 + dst, Mc + 2 * j);
+            const uint32_t col = smem_u32(b) + (uint32_t)(k >> 3) * F::LBO_B + (uint32_t)(k & 7) * 2;
+            const uint16_t* src = Mc + (long long)u0 * F::D + e;
+            for (int u = u0; u < F::D; u += rstep) {
+                cp_async_4(col + (uint32_t)(u >> 3) * F::SBO_B + (uint32_t)(u & 7) * 16, src);
+                src += rstep * F::D;
+            }
         }
         cp_async_wait_all();
     } else {
