@@ -82,7 +82,8 @@ WBMM_API wbmm_status wbmm_forward(const void *x, const void *T, void *y,
 /*
  * Bytes of device workspace wbmm_backward needs for the table gradient:
  * fp32 partial tables, one per (channel, fixed chunk of windows).  The chunk
- * split depends only on the shape, so dT is bit-identical from run to run.
+ * split depends only on the shape, the device's SM count and whether dX is
+ * computed in the same call, so dT is bit-identical from run to run.
  * Returns 0 for invalid shapes.
  */
 WBMM_API size_t wbmm_backward_workspace_bytes(int B, int C, int H, int W, int w, wbmm_dtype dt);
@@ -98,6 +99,10 @@ WBMM_API size_t wbmm_backward_workspace_bytes(int B, int C, int H, int W, int w,
  *   dT [C,(2w-1)^2] fp32, or NULL to skip it (overwritten, not accumulated)
  *   workspace: device buffer of at least wbmm_backward_workspace_bytes()
  *   bytes, 16-byte aligned; needed only when dT != NULL.
+ * With both outputs on a large enough bf16 problem the two gradient kernels
+ * run at the same time on disjoint SMs (dX on 2/5 of them); dT then sums in
+ * a different fixed order than a dT-only call, so the two differ by rounding
+ * (each deterministic).  The call's work is complete when its last kernel is.
  * Errors: as wbmm_forward, plus WORKSPACE.
  */
 WBMM_API wbmm_status wbmm_backward(const void *x, const void *T, const void *dY,
@@ -164,8 +169,9 @@ WBMM_API wbmm_status wbmm_dw3x3(const void *y, const void *K, void *z,
 
 /*
  * Table gradient for callers that cannot allocate device memory: the dT of
- * wbmm_backward (same kernels, same bits), with the fp32 partial tables kept
- * in a fixed 4 MiB array inside the library instead of a workspace argument.
+ * wbmm_backward called with dX = NULL (same kernels, same bits), with the
+ * fp32 partial tables kept in a fixed 4 MiB array inside the library instead
+ * of a workspace argument.
  * The paper has no counterpart to this entry point; it exists for hosts with a
  * fixed device-memory budget, plugins inside frameworks that own all device
  * allocations, and paths where cudaMalloc would synchronise the device.
