@@ -61,6 +61,32 @@ def test_forward_bf16_small(shape):
     check_bf16(to_np(y), ref, forward_rowbound(xr, Tr, w), "forward")
 
 
+# w = 28 on tensor cores (windows as the MMA's N dimension, a Toeplitz stack
+# of the table as A): one tile of 4 or 15 bands per channel (ragged), three
+# tiles per channel, and enough tiles that CTAs cross channel boundaries and
+# rebuild the stack (checked on sampled channels)
+BIG_SHAPES = [(2, 3, 56, 112, 28), (9, 2, 56, 112, 28), (5, 2, 84, 56, 28), (9, 60, 56, 112, 28)]
+
+
+@pytest.mark.parametrize("shape", BIG_SHAPES, ids=lambda s: "x".join(map(str, s)))
+def test_w28_forward_and_dx_tensor_cores(shape):
+    B, C, H, W, w = shape
+    x = gen((B, C, H, W), 33)
+    dy = gen((B, C, H, W), 34)
+    T = gen((C, (2 * w - 1) ** 2), 35, scale=0.02)
+    y = run_forward(x, T, w)
+    assert wb.wbmm_last_path() == 1, "tensor-core kernel expected"
+    dX, _ = wb.backward(x, T, dy, w, need_dt=False)
+    torch.cuda.synchronize()
+    assert wb.wbmm_get_device_status() == 0
+    assert wb.wbmm_last_path() == 1
+    cs = list(range(C)) if C <= 3 else [0, 1, C // 2, C - 2, C - 1]
+    xr, gr, Tr = to_np(x[:, cs]), to_np(dy[:, cs]), to_np(T[cs])
+    check_bf16(to_np(y[:, cs]), oracle.forward(xr, Tr, w), forward_rowbound(xr, Tr, w), "w28 y")
+    check_bf16(to_np(dX[:, cs]), oracle.backward_dx(gr, Tr, w),
+               forward_rowbound(gr, Tr[:, ::-1].copy(), w), "w28 dX")
+
+
 def test_forward_fp32_tiny_workload():
     wl = synth.WORKLOADS["tiny_fp32"]
     d = synth.draw(wl, seed=0)

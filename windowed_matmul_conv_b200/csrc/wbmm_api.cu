@@ -196,6 +196,12 @@ wbmm_status wbmm_forward(const void* x, const void* T, void* y, int B, int C, in
             t_last_path = 1;
         return st;
     }
+    if (dt == WBMM_BF16 && tc_big_supported(g)) {
+        st = from_cuda(tc_big_launch(g, kTable, x, T, y, L));
+        if (st == WBMM_OK)
+            t_last_path = 1;
+        return st;
+    }
     st = from_cuda(simt_fwd_launch(g, kTable, dt == WBMM_BF16, x, T, y, L));
     if (st == WBMM_OK)
         t_last_path = 2;
@@ -270,6 +276,9 @@ wbmm_status wbmm_backward(const void* x, const void* T, const void* dY, void* dX
             t_last_path = 1;
         } else if (dt == WBMM_BF16 && tc_fwd_supported(g, false)) {
             st = from_cuda(tc_fwd_launch(g, kTableFlip, dY, T, dX, nullptr, L));
+            t_last_path = 1;
+        } else if (dt == WBMM_BF16 && tc_big_supported(g)) {
+            st = from_cuda(tc_big_launch(g, kTableFlip, dY, T, dX, L));
             t_last_path = 1;
         } else {
             st = from_cuda(simt_fwd_launch(g, kTableFlip, dt == WBMM_BF16, dY, T, dX, L));

@@ -64,6 +64,13 @@ bool tc_toep_supported(const Geom& g);
 cudaError_t tc_toep_launch(const Geom& g, AMode mode, const void* x, const void* T, void* y,
                            const Launch& L);
 
+// tcgen05 forward / input gradient for w = 28 from the table, windows as the
+// MMA's N dimension and a per-channel Toeplitz stack as A (mode kTable or
+// kTableFlip only).
+bool tc_big_supported(const Geom& g);
+cudaError_t tc_big_launch(const Geom& g, AMode mode, const void* x, const void* T, void* y,
+                          const Launch& L);
+
 // tcgen05 forward with a cached [C][d][d] matrix, windows as the MMA's M
 // dimension (no fused 3x3).
 bool tc_cached_supported(const Geom& g);
