@@ -18,21 +18,23 @@
 //
 // starting at row 128m + (w - 1 - r)*32: Q (two halves, 110 KB at w = 28) is
 // built in shared memory once per channel and only the descriptors' start
-// addresses move.  The B operand is 32 windows of one channel (K-major, 16-
+// addresses move.  The B operand is 64 windows of one channel (K-major, 16-
 // slot K steps), produced four window rows at a time: the producer copies the
 // four image rows of every band of the tile with bulk copies, the transform
 // rearranges them into the K-major layout (zeros beyond w), and the MMA warp
-// runs the 7 x 8 MMAs of the chunk (M = 128, N = 32, K = 16) into a TMEM
-// accumulator of 7 x 32 columns (two of them, so a tile's epilogue overlaps
-// the next tile's MMAs).  The epilogue reads one output row per warp lane
-// quarter (lane = q, 32 registers = 32 windows) and stores bf16 straight to
-// the output map: 28 consecutive elements per warp store.
+// runs the 7 x 8 MMAs of the chunk (M = 128, N = 64, K = 16) into a TMEM
+// accumulator of 7 x 64 columns.  Each MMA reads its 4 KB A block from shared
+// memory, so N = 64 (not 32) keeps the tensor core's operand reads from
+// bounding it.  The epilogue reads one output row per warp lane quarter
+// (lane = q, 32 registers = 32 windows, two loads) and stores bf16 straight
+// to the output map: 28 consecutive elements per warp store.
 //
-// Warp roles (448 threads):
+// Warp roles (576 threads):
 //   warp 0       producer: bulk copies of four-row chunks into a raw ring
 //   warp 1       MMA issuer (one thread) and TMEM owner
-//   warps 2..5   transform: raw chunk -> B chunk (thread = window, row)
-//   warps 6..13  epilogue, and Q for each channel (after the channel's last
+//   warps 2..9   transform: raw chunk -> B chunk (thread = window, row);
+//                after a tile's chunks, half of the accumulator drain
+//   warps 10..17 epilogue, and Q for each channel (after the channel's last
 //                accumulator is complete, so no MMA still reads the old Q)
 // Every wait is bounded; a wait that runs out raises the CTA's abort flag and
 // the device status word, and every role then runs its loop without doing
@@ -51,7 +53,7 @@ struct BigCfg {
     static constexpr int L = 2 * WS - 1;
     static constexpr int TSZ = L * L;
     static constexpr int MT = (WS * RP + 127) / 128;         // 128-row M tiles
-    static constexpr int NW = 32;                            // windows per tile (MMA N)
+    static constexpr int NW = 64;                            // windows per tile (MMA N)
     static constexpr int CR = 4;                             // window rows per chunk
     static constexpr int NCH = (WS + CR - 1) / CR;           // chunks per tile
     static constexpr int KCH = CR * 2;                       // K steps per chunk
@@ -60,17 +62,19 @@ struct BigCfg {
     static constexpr uint32_t KSTEP_BYTES = (NW / 8) * 256;  // one K step of B
     static constexpr uint32_t BCH_BYTES = KCH * KSTEP_BYTES; // one chunk of B
     static constexpr uint32_t IDESC = idesc_bf16(128, NW);
-    static_assert(MT * NW <= 256, "two accumulators fit in TMEM");
+    static_assert(MT * NW <= 512, "the accumulator fits in TMEM");
     static_assert(QROWS % 8 == 0 && ((WS - 1) * RP) % 8 == 0, "Q rows in whole core matrices");
 };
 
 constexpr int kBigRawRing = 8;
 constexpr int kBigBRing = 3;
 constexpr int kBigXformWarp0 = 2;
-constexpr int kBigXformWarps = 4;
+constexpr int kBigXformWarps = 8;
 constexpr int kBigEpiWarp0 = kBigXformWarp0 + kBigXformWarps;
 constexpr int kBigEpiWarps = 8;
 constexpr int kBigThreads = (kBigEpiWarp0 + kBigEpiWarps) * 32;
+// warps that drain the accumulator: the epilogue's and the transform's
+constexpr int kBigEpilogueThreads = (kBigEpiWarps + kBigXformWarps) * 32;
 
 struct TcBigParams {
     const uint16_t* x;      // bf16 bits, [B][C][H][W]
@@ -151,6 +155,39 @@ __device__ __forceinline__ void big_build_q(uint8_t* q, const uint16_t* tst, int
     }
 }
 
+// Output rows of M tiles idx, idx + 4, ... of the tile in the accumulator:
+// the warp's lane quarter holds output row p = 4m + quarter and lane q its
+// column; the accumulator's NW columns are the tile's windows (wb: their
+// output bases).  Stores bf16 straight to y, 28 consecutive elements per
+// warp store.
+template <int WS>
+__device__ __forceinline__ void big_drain(const TcBigParams& P, uint32_t tmem, int quarter,
+                                          int lane, int idx, int nwin, const long long* wb)
+{
+    using F = BigCfg<WS>;
+#pragma unroll 1
+    for (int m = idx; m < F::MT; m += 4) {
+        const int p = 4 * m + quarter;
+        if (p >= WS)
+            continue;
+        const long long off = (long long)p * P.W + lane;
+#pragma unroll 1
+        for (int g32 = 0; g32 < F::NW / 32; ++g32) {
+            uint32_t r[32];
+            tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(m * F::NW + g32 * 32),
+                      r);
+            tmem_wait_ld(r);
+            if (lane >= WS)
+                continue;
+#pragma unroll
+            for (int nn = 0; nn < 32; ++nn)
+                if (g32 * 32 + nn < nwin)
+                    P.y[wb[g32 * 32 + nn] + off] =
+                        __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(r[nn])));
+        }
+    }
+}
+
 template <int WS, int MODE>
 __global__ void __launch_bounds__(kBigThreads, 1)
     wbmm_tc_big_kernel(const __grid_constant__ TcBigParams P)
@@ -182,7 +219,7 @@ __global__ void __launch_bounds__(kBigThreads, 1)
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&S.acc_full[i], 1);
-            mbar_init(&S.acc_empty[i], kBigEpiWarps);
+            mbar_init(&S.acc_empty[i], kBigEpiWarps + kBigXformWarps);
         }
         mbar_init(&S.q_full, kBigEpiWarps);
         mbar_init(&S.fin, 1);
@@ -249,15 +286,14 @@ __global__ void __launch_bounds__(kBigThreads, 1)
                     cur_c = t.c;
                     ++ci;
                 }
-                const int a = seq & 1;
                 bool ok = !*abort;
                 if (first)
                     ok = ok && mbar_wait(&S.q_full, ci & 1, abort, P.budget, P.status);
-                if (seq >= 2)
-                    ok = ok && mbar_wait(&S.acc_empty[a], ((seq >> 1) - 1) & 1, abort, P.budget,
+                if (seq >= 1)
+                    ok = ok && mbar_wait(&S.acc_empty[0], (seq - 1) & 1, abort, P.budget,
                                          P.status);
                 const uint32_t q0 = smem_u32(q_base);
-                const uint32_t d0 = tmem + (uint32_t)(a * 256);
+                const uint32_t d0 = tmem;
                 for (int ch = 0; ch < F::NCH; ++ch) {
                     const int ss = seq * F::NCH + ch, bs = ss % kBigBRing;
                     ok = ok && mbar_wait(&S.b_full[bs], (ss / kBigBRing) & 1, abort, P.budget,
@@ -285,7 +321,7 @@ __global__ void __launch_bounds__(kBigThreads, 1)
                     tc_commit(&S.b_empty[bs]);
                 }
                 if (ok)
-                    tc_commit(&S.acc_full[a]);
+                    tc_commit(&S.acc_full[0]);
             }
             tc_commit(&S.fin);
             mbar_wait_drain(&S.fin, 0, P.budget, P.status);
@@ -296,7 +332,7 @@ __global__ void __launch_bounds__(kBigThreads, 1)
         // that row as two pairs of 16-byte core-matrix rows (zeros past w and
         // for windows past the tile's last band).
         const int tid = threadIdx.x - kBigXformWarp0 * 32;
-        const int n = tid & 31, rr = tid >> 5;
+        const int n = tid % F::NW, rr = tid / F::NW;
         for (int seq = 0; seq < n_it; ++seq) {
             const BandTile t = big_tile(P, it0 + seq);
             const int nwin = t.nb * P.nw;
@@ -338,13 +374,25 @@ __global__ void __launch_bounds__(kBigThreads, 1)
                     mbar_arrive(&S.raw_empty[s]);
                 }
             }
+            // then take two of the four warps per lane quarter that drain
+            // this tile's accumulator (the MMAs of the next tile wait for it)
+            named_bar_sync(3, kBigEpilogueThreads);       // window bases written
+            bool ok = !*abort;
+            ok = ok && mbar_wait(&S.acc_full[0], seq & 1, abort, P.budget, P.status);
+            ok = __all_sync(0xffffffffu, ok);
+            tc_fence_after();
+            if (ok)
+                big_drain<WS>(P, tmem, warp & 3, lane, 2 + ((warp - kBigXformWarp0) >> 2), nwin,
+                              wbase + (seq & 1) * F::NW);
+            tc_fence_before();
+            __syncwarp();
+            if (ok && lane == 0)
+                mbar_arrive(&S.acc_empty[0]);
         }
     } else {
         // ------------------------------------------------------ epilogue
-        // Two warps per TMEM lane quarter; warp half hf takes M tiles hf,
-        // hf+2, ...  In M tile m, quarter qt holds output row p = 4m + qt and
-        // lane q its column: the 32 accumulator columns are the tile's 32
-        // windows.
+        // Two warps per TMEM lane quarter, with the transform's two: warp
+        // half hf drains M tiles hf, hf+4 (big_drain).
         const int quarter = warp & 3;
         const int hf = (warp - kBigEpiWarp0) >> 2;
         const int et = threadIdx.x - kBigEpiWarp0 * 32;
@@ -370,7 +418,7 @@ __global__ void __launch_bounds__(kBigThreads, 1)
         for (int seq = 0; seq < n_it; ++seq) {
             const BandTile t = big_tile(P, it0 + seq);
             const int nwin = t.nb * P.nw;
-            const int a = seq & 1;
+            const int a = seq & 1;          // window-base buffer
             // output base of each window of the tile (row 0, column 0)
             if (et < F::NW) {
                 long long v = 0;
@@ -380,33 +428,17 @@ __global__ void __launch_bounds__(kBigThreads, 1)
                 }
                 wbase[a * F::NW + et] = v;
             }
-            named_bar_sync(3, EPT);
+            named_bar_sync(3, kBigEpilogueThreads);
             bool ok = !*abort;
-            ok = ok && mbar_wait(&S.acc_full[a], (seq >> 1) & 1, abort, P.budget, P.status);
+            ok = ok && mbar_wait(&S.acc_full[0], seq & 1, abort, P.budget, P.status);
             ok = __all_sync(0xffffffffu, ok);
             tc_fence_after();
-#pragma unroll 1
-            for (int m = hf; m < F::MT; m += 2) {
-                const int p = 4 * m + quarter;
-                if (!ok || p >= WS)
-                    continue;
-                uint32_t r[32];
-                tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(a * 256 + m * F::NW),
-                          r);
-                tmem_wait_ld(r);
-                if (lane >= WS)
-                    continue;
-                const long long off = (long long)p * P.W + lane;
-#pragma unroll
-                for (int nn = 0; nn < F::NW; ++nn)
-                    if (nn < nwin)
-                        P.y[wbase[a * F::NW + nn] + off] =
-                            __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(r[nn])));
-            }
+            if (ok)
+                big_drain<WS>(P, tmem, quarter, lane, hf, nwin, wbase + a * F::NW);
             tc_fence_before();
             __syncwarp();
             if (ok && lane == 0)
-                mbar_arrive(&S.acc_empty[a]);
+                mbar_arrive(&S.acc_empty[0]);
             // the channel's last tile is complete (acc_full): no MMA reads Q
             if (seq + 1 < n_it && big_tile(P, it0 + seq + 1).c != t.c)
                 build_for(big_tile(P, it0 + seq + 1).c);
