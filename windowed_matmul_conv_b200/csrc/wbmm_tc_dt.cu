@@ -7,7 +7,8 @@
 //   dT[(p-r+w-1)(2w-1) + (q-s+w-1)] = sum over (u=(p,q), v=(r,s)) of G[u, v].
 //
 // The channels' tiles, in channel order, are split into one contiguous,
-// balanced range per CTA.  A segment is the part of a CTA's range inside one
+// balanced range per CTA: of whole channels when that gives no CTA more tiles
+// than a split at tile granularity, else of tiles.  A segment is the part of a CTA's range inside one
 // channel; each segment ends with one reduction of G into its own fp32 partial
 // table, at index c + k (channel c, CTA k: ranges are ordered, so the index
 // is unique).  A channel inside one CTA's range is written to dT directly.
@@ -105,7 +106,8 @@ struct TcDtParams {
     int bpt;
     int tpc;                // tiles per channel
     int bands;
-    int rq, rr;             // range split: CTA k gets rq + (k < rr) tiles
+    int rq, rr;             // range split: CTA k gets rq + (k < rr) units
+    int unit;               // tiles per unit: 1, or tpc (whole channels)
     int dep_wait;           // 1: wait for the previous kernel before any load;
                             // 0: the previous kernel is the same call's input
                             // gradient, which writes nothing this one touches,
@@ -140,16 +142,17 @@ struct DtTile {
 // The CTA whose range holds tile t (inverse of dt_range).
 __device__ __forceinline__ int dt_cta_of(const TcDtParams& P, long long t)
 {
+    const long long u = t / P.unit;
     const long long big = (long long)P.rr * (P.rq + 1);
-    return (int)(t < big ? t / (P.rq + 1) : P.rr + (t - big) / P.rq);
+    return (int)(u < big ? u / (P.rq + 1) : P.rr + (u - big) / P.rq);
 }
 
 // The tile range of a CTA: [t0, t1) of the channel-major tile sequence.
 __device__ __forceinline__ void dt_range(const TcDtParams& P, int& t0, int& t1)
 {
     const int k = (int)blockIdx.x;
-    t0 = k * P.rq + (k < P.rr ? k : P.rr);
-    t1 = t0 + P.rq + (k < P.rr ? 1 : 0);
+    t0 = (k * P.rq + (k < P.rr ? k : P.rr)) * P.unit;
+    t1 = t0 + (P.rq + (k < P.rr ? 1 : 0)) * P.unit;
 }
 
 // Every role walks the CTA's range in the same order.
@@ -701,8 +704,20 @@ cudaError_t dt_launch_ws(const Geom& g, const void* x, const void* dy, float* wo
         grid = tiles;
     if (grid < 1)
         return cudaSuccess;
-    P.rq = tiles / grid;
-    P.rr = tiles - P.rq * grid;
+    // Ranges of whole channels when that costs a CTA no more tiles than the
+    // tile-granular split (no channel is then shared between CTAs: one
+    // reduction of G per channel, no partial tables), else tile ranges.
+    const int per_tile = (tiles + grid - 1) / grid;
+    const int per_chan = (g.C + grid - 1) / grid * P.tpc;
+    if (g.C >= grid && per_chan <= per_tile) {
+        P.unit = P.tpc;
+        P.rq = g.C / grid;
+        P.rr = g.C - P.rq * grid;
+    } else {
+        P.unit = 1;
+        P.rq = tiles / grid;
+        P.rr = tiles - P.rq * grid;
+    }
     P.dep_wait = after_dx ? 0 : 1;
     P.use_tmap = 0;
     P.kimg = 0;
