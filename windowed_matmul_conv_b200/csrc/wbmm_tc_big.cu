@@ -155,36 +155,38 @@ __device__ __forceinline__ void big_build_q(uint8_t* q, const uint16_t* tst, int
     }
 }
 
-// Output rows of M tiles idx, idx + 4, ... of the tile in the accumulator:
-// the warp's lane quarter holds output row p = 4m + quarter and lane q its
-// column; the accumulator's NW columns are the tile's windows (wb: their
-// output bases).  Stores bf16 straight to y, 28 consecutive elements per
-// warp store.
+// Windows 16*idx .. 16*idx+15 of the tile, every output row of the warp's
+// lane quarter: in M tile m the quarter holds output row p = 4m + quarter,
+// lane q its column, and accumulator columns m*NW + n are window n (wb: the
+// windows' output bases, read once).  Stores bf16 straight to y, 28
+// consecutive elements per warp store.
 template <int WS>
 __device__ __forceinline__ void big_drain(const TcBigParams& P, uint32_t tmem, int quarter,
                                           int lane, int idx, int nwin, const long long* wb)
 {
     using F = BigCfg<WS>;
+    const int n0 = 16 * idx;
+    if (n0 >= nwin)
+        return;
+    long long base[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+        base[i] = wb[n0 + i] + lane;
 #pragma unroll 1
-    for (int m = idx; m < F::MT; m += 4) {
+    for (int m = 0; m < F::MT; ++m) {
         const int p = 4 * m + quarter;
         if (p >= WS)
+            break;
+        uint32_t r[16];
+        tmem_ld16(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(m * F::NW + n0), r);
+        tmem_wait_ld(r);
+        if (lane >= WS)
             continue;
-        const long long off = (long long)p * P.W + lane;
-#pragma unroll 1
-        for (int g32 = 0; g32 < F::NW / 32; ++g32) {
-            uint32_t r[32];
-            tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(m * F::NW + g32 * 32),
-                      r);
-            tmem_wait_ld(r);
-            if (lane >= WS)
-                continue;
+        const long long off = (long long)p * P.W;
 #pragma unroll
-            for (int nn = 0; nn < 32; ++nn)
-                if (g32 * 32 + nn < nwin)
-                    P.y[wb[g32 * 32 + nn] + off] =
-                        __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(r[nn])));
-        }
+        for (int i = 0; i < 16; ++i)
+            if (n0 + i < nwin)
+                P.y[base[i] + off] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(r[i])));
     }
 }
 
@@ -375,7 +377,8 @@ __global__ void __launch_bounds__(kBigThreads, 1)
                 }
             }
             // then take two of the four warps per lane quarter that drain
-            // this tile's accumulator (the MMAs of the next tile wait for it)
+            // this tile's accumulator (windows 32 .. 63; the MMAs of the next
+            // tile wait for it)
             named_bar_sync(3, kBigEpilogueThreads);       // window bases written
             bool ok = !*abort;
             ok = ok && mbar_wait(&S.acc_full[0], seq & 1, abort, P.budget, P.status);
@@ -392,7 +395,7 @@ __global__ void __launch_bounds__(kBigThreads, 1)
     } else {
         // ------------------------------------------------------ epilogue
         // Two warps per TMEM lane quarter, with the transform's two: warp
-        // half hf drains M tiles hf, hf+4 (big_drain).
+        // half hf drains windows 16hf .. 16hf+15 (big_drain).
         const int quarter = warp & 3;
         const int hf = (warp - kBigEpiWarp0) >> 2;
         const int et = threadIdx.x - kBigEpiWarp0 * 32;
