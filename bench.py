@@ -136,10 +136,9 @@ class ClockSampler:
 
     def start(self):
         try:
-            out_dir = os.path.join(ROOT, "gpurun_out")
-            os.makedirs(out_dir, exist_ok=True)
-            self.path = os.path.join(out_dir, "clocks_rank%d.csv" % self.gpu)
-            self.fh = open(self.path, "w")
+            import tempfile
+            fd, self.path = tempfile.mkstemp(prefix="wbmm_clocks_gpu%d_" % self.gpu, suffix=".csv")
+            self.fh = os.fdopen(fd, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
                  "--format=csv,noheader,nounits", "-lms", "100"],
@@ -171,6 +170,10 @@ class ClockSampler:
             for nm, v in zip(names, parts[5:9]):
                 if v.lower() == "active":
                     reasons.add(nm)
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
         if not sm:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
