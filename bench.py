@@ -5,7 +5,9 @@ synthetic input.  Default workload (the training step): B128 C256 28x28, w=14,
 bf16 -- forward y = WBMM(x; T), then the backward dX = M^T dY and the table
 gradient dT, all through the C ABI.  Other workloads (--workload): fwd
 (B64 C128 56x56 w14), sweep7 / sweep14 / sweep28 (B32 C256 112x112), cached
-(B8 C96 224x224 w14, cached matrices + 3x3 mixing).
+(B8 C96 224x224 w14, cached matrices + 3x3 mixing), fwd32 (the fp32 forward
+of the fwd shape) and reparam (the cached shape through one matrix merged from a
+14x14 and a 7x7 table).
 
 Multi-GPU (torchrun): every rank owns its own block of channels with the
 per-GPU workload above (weak scaling); channels are independent, so the hot
@@ -13,7 +15,7 @@ path has no collective.  Timing is device time (CUDA events) with a barrier on
 both sides, max over ranks.
 
 --impl reference runs the fp64 CPU oracle on the host cores instead (bounded
-sample per step); it is the slow baseline the driver divides by.
+sample per step), a deliberately slow comparison arm with the same JSON line.
 """
 import argparse
 import json
