@@ -92,3 +92,98 @@ def test_status_strings(lib):
     f.argtypes = [ctypes.c_int]
     for s in range(9):
         assert f(s).decode().startswith("WBMM_")
+
+
+def _proto(lib, name, argtypes):
+    f = getattr(lib, name)
+    f.restype = ctypes.c_int
+    f.argtypes = argtypes
+    return f
+
+
+P, I, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+
+# Addresses that are never dereferenced: every call below must be rejected by
+# the host-side checks, before any device call.  Blocks are 256 MB apart so
+# that buffers of the shapes used never overlap unless a test says so.
+A0, A1, A2, A3, A4 = (0x10000000 * k for k in (1, 2, 3, 4, 5))
+
+
+def test_backward_argument_checks(lib):
+    f = _proto(lib, "wbmm_backward", [P, P, P, P, P, P, S] + [I] * 6 + [P])
+    ws = lib.wbmm_backward_workspace_bytes
+    ws.restype, ws.argtypes = S, [I] * 6
+    need = ws(2, 4, 28, 28, 14, 1)
+    assert need > 0
+
+    def call(x=A0, T=A1, dY=A2, dX=A3, dT=A4, work=A4 + 0x100000, nbytes=need,
+             shape=(2, 4, 28, 28, 14), dt=1):
+        return f(x, T, dY, dX, dT, work, nbytes, *shape, dt, None)
+
+    assert call(dt=2) == 3                               # dtype
+    assert call(dY=None) == 1                            # dY is required
+    assert call(T=None) == 1                             # dX needs the table
+    assert call(x=None) == 1                             # dT needs the input
+    assert call(shape=(2, 4, 28, 30, 14)) == 2           # W % w
+    assert call(shape=(2, 4, 28, 28, 0)) == 1            # w = 0
+    assert call(shape=(2, 4, 130, 130, 65)) == 5         # w beyond limit
+    assert call(dX=A3 + 8) == 4                          # bf16 maps need 16 B
+    assert call(dT=A4 + 2) == 4                          # dT is fp32
+    assert call(dX=A2 + 64) == 1                         # dX overlaps dY
+    assert call(dT=A0 + 64) == 1                         # dT overlaps x
+    assert call(work=None) == 6                          # dT needs a workspace
+    assert call(nbytes=need - 4) == 6                    # ... of the stated size
+    assert call(work=A4 + 0x100008) == 4                 # ... 16-byte aligned
+    assert call(work=A4 + 64) == 1                       # ... not overlapping dT
+    assert call(work=A2 + 64) == 1                       # ... nor dY
+    # dX only: neither x nor a workspace is needed, so the first failing check
+    # is the misaligned dX
+    assert call(dT=None, x=None, work=None, nbytes=0, dX=A3 + 8) == 4
+    # dT only: no table needed
+    assert call(dX=None, T=None, dT=A4 + 2) == 4
+
+
+def test_cache_and_merge_argument_checks(lib):
+    cache = _proto(lib, "wbmm_cache_matrices", [P, P, I, I, I, P])
+    assert cache(A0, A1, 4, 14, 3, None) == 3
+    assert cache(None, A1, 4, 14, 1, None) == 1
+    assert cache(A0, A1, 0, 14, 1, None) == 1
+    assert cache(A0, A1, 4, 65, 1, None) == 5
+    assert cache(A0, A1 + 2, 4, 14, 1, None) == 4
+    assert cache(A0, A0 + 128, 4, 14, 1, None) == 1      # M overlaps T
+    merge = _proto(lib, "wbmm_reparam_merge", [P, P, P, I, I, I, I, P])
+    assert merge(A0, A1, A2, 4, 14, 7, 5, None) == 3
+    assert merge(A0, None, A2, 4, 14, 7, 1, None) == 1
+    assert merge(A0, A1, A2, 4, 14, 5, 1, None) == 1     # k must divide w
+    assert merge(A0, A1, A2, 4, 14, 0, 1, None) == 1
+    assert merge(A0, A1, A2, 4, 70, 7, 1, None) == 5
+    assert merge(A0, A1, A2 + 8, 4, 14, 7, 1, None) == 4
+    assert merge(A0, A2 + 64, A2, 4, 14, 7, 1, None) == 1  # M overlaps the small table
+
+
+def test_cached_and_dw_argument_checks(lib):
+    fc = _proto(lib, "wbmm_forward_cached", [P, P, P, P] + [I] * 6 + [P])
+    assert fc(A0, A1, None, A2, 1, 4, 28, 28, 14, 4, None) == 3
+    assert fc(A0, None, None, A2, 1, 4, 28, 28, 14, 1, None) == 1
+    assert fc(A0, A1, None, A2, 1, 4, 28, 21, 14, 1, None) == 2
+    assert fc(A0, A1, A3 + 2, A2, 1, 4, 28, 28, 14, 1, None) == 4   # 3x3 weights
+    assert fc(A0, A1, None, A0 + 16, 1, 4, 28, 28, 14, 1, None) == 1  # out overlaps x
+    assert fc(A0, A1, A2 + 16, A2, 1, 4, 28, 28, 14, 1, None) == 1  # out overlaps the weights
+    dw = _proto(lib, "wbmm_dw3x3", [P, P, P] + [I] * 5 + [P])
+    assert dw(A0, A1, A2, 1, 4, 9, 13, 7, None) == 3
+    assert dw(A0, A1, None, 1, 4, 9, 13, 1, None) == 1
+    assert dw(A0, A1, A2, 1, 4, 0, 13, 1, None) == 1
+    assert dw(A0 + 8, A1, A2, 1, 4, 9, 13, 1, None) == 4
+    assert dw(A0, A1, A0 + 32, 1, 4, 9, 13, 1, None) == 1           # in place is refused
+
+
+def test_static_table_gradient_argument_checks(lib):
+    f = _proto(lib, "wbmm_backward_dt_static", [P, P, P] + [I] * 6 + [P])
+    assert f(A0, A1, A2, 2, 4, 28, 28, 14, 2, None) == 3
+    assert f(A0, None, A2, 2, 4, 28, 28, 14, 1, None) == 1
+    assert f(A0, A1, A2, 2, 4, 28, 27, 14, 1, None) == 2
+    assert f(A0, A1, A2, 2, 4, 130, 130, 65, 1, None) == 5
+    assert f(A0, A1 + 8, A2, 2, 4, 28, 28, 14, 1, None) == 4
+    assert f(A0, A1, A0 + 64, 2, 4, 28, 28, 14, 1, None) == 1       # dT overlaps x
+    # more partial tables than the 4 MiB static array holds
+    assert f(A0, A1, A2, 1, 2048, 14, 14, 14, 1, None) == 6
