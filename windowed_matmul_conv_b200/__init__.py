@@ -5,6 +5,10 @@ Each ``wbmm_*`` function has the name and meaning of the C entry point in
 ``include/wbmm.h`` and only marshals arguments: shapes and dtypes come from
 the torch tensors, device pointers from ``data_ptr()``, the stream from
 ``torch.cuda.current_stream()``.  A non-zero status raises ``WbmmError``.
+Plain pointers carry no sizes, so before the call the binding checks what
+the library cannot: every buffer is on the current device, has the call's
+dtype (fp32 for dT) and holds at least the elements the call reads or writes
+(``WbmmError`` with ``WBMM_ERR_DTYPE`` or ``WBMM_ERR_INVALID_ARG``).
 PyTorch is used for device memory and streams; every step of the operator
 runs in the library's CUDA kernels.  Importing this package fails loudly if
 the library has not been built (``python windowed_matmul_conv_b200/build.py``).
@@ -62,10 +66,14 @@ for _f in ("wbmm_forward", "wbmm_backward", "wbmm_backward_dt_static", "wbmm_cac
     getattr(_lib, _f).restype = _i
 
 
+WBMM_ERR_INVALID_ARG, WBMM_ERR_DTYPE = 1, 3
+
+
 class WbmmError(RuntimeError):
-    def __init__(self, status):
+    def __init__(self, status, detail=None):
         self.status = status
-        super().__init__(_lib.wbmm_status_string(status).decode())
+        msg = _lib.wbmm_status_string(status).decode()
+        super().__init__(msg if detail is None else "%s: %s" % (msg, detail))
 
 
 def _check(status):
@@ -89,9 +97,38 @@ def _p(t):
     return ctypes.c_void_p(t.data_ptr())
 
 
-def _stream(stream):
+def _stream(stream, ref=None):
+    """Stream handle for a call whose maps live on ``ref``'s device.  The
+    library launches on the current device, so ``ref`` and the stream must
+    be on it."""
     s = torch.cuda.current_stream() if stream is None else stream
+    if ref is not None:
+        d, cur = ref.get_device(), torch.cuda.current_device()
+        if d != cur or s.device_index != d:
+            raise WbmmError(WBMM_ERR_INVALID_ARG,
+                            "maps on cuda:%d, stream on cuda:%d, current device cuda:%d"
+                            % (d, s.device_index, cur))
     return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(name, t, numel, ref, dtype=None):
+    """Buffer ``t`` (optional) must sit on ``ref``'s device, have ``ref``'s
+    dtype (or ``dtype``) and hold at least ``numel`` elements."""
+    want = dtype or ref.dtype
+    if t is None or (t.dtype is want and t.numel() >= numel
+                     and t.get_device() == ref.get_device()):
+        return
+    if t.get_device() != ref.get_device():
+        raise WbmmError(WBMM_ERR_INVALID_ARG, "%s is on %s, the map on %s"
+                        % (name, t.device, ref.device))
+    if t.dtype is not want:
+        raise WbmmError(WBMM_ERR_DTYPE, "%s is %s, the call needs %s" % (name, t.dtype, want))
+    raise WbmmError(WBMM_ERR_INVALID_ARG, "%s holds %d elements, the call needs %d"
+                    % (name, t.numel(), numel))
+
+
+def _tsz(w):
+    return (2 * int(w) - 1) ** 2
 
 
 def _map_shape(x):
@@ -104,42 +141,62 @@ def _map_shape(x):
 
 def wbmm_forward(x, T, y, w, stream=None):
     B, C, H, W = _map_shape(x)
-    _check(_lib.wbmm_forward(_p(x), _p(T), _p(y), B, C, H, W, int(w), _dt(x), _stream(stream)))
+    _need("T", T, C * _tsz(w), x)
+    _need("y", y, x.numel(), x)
+    _check(_lib.wbmm_forward(_p(x), _p(T), _p(y), B, C, H, W, int(w), _dt(x),
+                             _stream(stream, x)))
 
 
 def wbmm_backward_workspace_bytes(B, C, H, W, w, dtype):
-    dt = WBMM_BF16 if dtype == torch.bfloat16 else WBMM_F32
+    dt = _dt(torch.empty(0, dtype=dtype))
     return int(_lib.wbmm_backward_workspace_bytes(B, C, H, W, int(w), dt))
 
 
 def wbmm_backward(x, T, dY, dX, dT, workspace, w, stream=None):
     B, C, H, W = _map_shape(dY)
+    _need("x", x, dY.numel(), dY)
+    _need("T", T, C * _tsz(w), dY)
+    _need("dX", dX, dY.numel(), dY)
+    _need("dT", dT, C * _tsz(w), dY, torch.float32)
+    if workspace is not None and workspace.get_device() != dY.get_device():
+        raise WbmmError(WBMM_ERR_INVALID_ARG, "workspace is on %s, the map on %s"
+                        % (workspace.device, dY.device))
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(_lib.wbmm_backward(_p(x), _p(T), _p(dY), _p(dX), _p(dT), _p(workspace), ws_bytes,
-                              B, C, H, W, int(w), _dt(dY), _stream(stream)))
+                              B, C, H, W, int(w), _dt(dY), _stream(stream, dY)))
 
 
 def wbmm_backward_dt_static(x, dY, dT, w, stream=None):
     """dT of wbmm_backward with the library's fixed scratch array (no allocation)."""
     B, C, H, W = _map_shape(dY)
+    _need("x", x, dY.numel(), dY)
+    _need("dT", dT, C * _tsz(w), dY, torch.float32)
     _check(_lib.wbmm_backward_dt_static(_p(x), _p(dY), _p(dT), B, C, H, W, int(w), _dt(dY),
-                                        _stream(stream)))
+                                        _stream(stream, dY)))
 
 
 def wbmm_cache_matrices(T, M, w, stream=None):
-    _check(_lib.wbmm_cache_matrices(_p(T), _p(M), int(T.shape[0]), int(w), _dt(T),
-                                    _stream(stream)))
+    """T: [C, (2w-1)^2]; M: [C, w*w, w*w]."""
+    C = int(T.shape[0])
+    _need("T", T, C * _tsz(w), T)
+    _need("M", M, C * int(w) ** 4, T)
+    _check(_lib.wbmm_cache_matrices(_p(T), _p(M), C, int(w), _dt(T), _stream(stream, T)))
 
 
 def wbmm_forward_cached(x, M, dw3x3, out, w, stream=None):
     B, C, H, W = _map_shape(x)
+    _need("M", M, C * int(w) ** 4, x)
+    _need("dw3x3", dw3x3, C * 9, x)
+    _need("out", out, x.numel(), x)
     _check(_lib.wbmm_forward_cached(_p(x), _p(M), _p(dw3x3), _p(out), B, C, H, W, int(w),
-                                    _dt(x), _stream(stream)))
+                                    _dt(x), _stream(stream, x)))
 
 
 def wbmm_dw3x3(y, K, z, stream=None):
     B, C, H, W = _map_shape(y)
-    _check(_lib.wbmm_dw3x3(_p(y), _p(K), _p(z), B, C, H, W, _dt(y), _stream(stream)))
+    _need("K", K, C * 9, y)
+    _need("z", z, y.numel(), y)
+    _check(_lib.wbmm_dw3x3(_p(y), _p(K), _p(z), B, C, H, W, _dt(y), _stream(stream, y)))
 
 
 def wbmm_get_device_status(stream=None):
@@ -188,8 +245,13 @@ def backward(x, T, dY, w, need_dx=True, need_dt=True, stream=None):
 
 
 def wbmm_reparam_merge(Tw, Tk, M, w, k, stream=None):
-    _check(_lib.wbmm_reparam_merge(_p(Tw), _p(Tk), _p(M), int(Tw.shape[0]), int(w), int(k),
-                                   _dt(Tw), _stream(stream)))
+    """Tw: [C, (2w-1)^2]; Tk: [C, (2k-1)^2]; M: [C, w*w, w*w]."""
+    C = int(Tw.shape[0])
+    _need("Tw", Tw, C * _tsz(w), Tw)
+    _need("Tk", Tk, C * _tsz(k), Tw)
+    _need("M", M, C * int(w) ** 4, Tw)
+    _check(_lib.wbmm_reparam_merge(_p(Tw), _p(Tk), _p(M), C, int(w), int(k), _dt(Tw),
+                                   _stream(stream, Tw)))
 
 
 def reparam_merge(Tw, Tk, w, k, stream=None):
