@@ -355,6 +355,36 @@ def cpu_baseline(wl, host, budget_s=10.0):
                       % (bs, wl.B, wl.C, runs, el)}
 
 
+def dw5x5_context(sets, K, stream):
+    """Same-run context, not part of the step: torch's depthwise 5x5
+    convolution (padding 2, library kernel) on the step's input maps, the
+    baseline the pages compare WBMM with.  Never raises: a failure is
+    reported in the returned record."""
+    rec = {"op": "torch conv2d, 5x5 depthwise (groups=C), padding 2, on the step's x"}
+    try:
+        xs = [s["x"] for s in sets]
+        C = xs[0].shape[1]
+        g = torch.Generator(device="cpu")
+        g.manual_seed(5)
+        wgt = (torch.randn((C, 1, 5, 5), generator=g) * 0.2).to(xs[0].dtype).to(xs[0].device)
+        with torch.no_grad():
+            for k in range(3):
+                torch.nn.functional.conv2d(xs[k % len(xs)], wgt, padding=2, groups=C)
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for k in range(K):
+                torch.nn.functional.conv2d(xs[k % len(xs)], wgt, padding=2, groups=C)
+            b.record(stream)
+            torch.cuda.synchronize()
+        us = a.elapsed_time(b) / K * 1e3
+        nbytes = 2 * xs[0].numel() * xs[0].element_size()
+        rec.update({"us": round(us, 2), "gbs": round(nbytes / (us * 1e-6) / 1e9, 1)})
+    except Exception as e:   # context only: never costs the benchmark line
+        rec["unavailable"] = ("%s: %s" % (type(e).__name__, e))[:200]
+    return rec
+
+
 def run_gpu(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
@@ -487,6 +517,8 @@ def run_gpu(args, rank, world, local_rank):
     barrier(world)
     e2e_ms = max_over_ranks(f0.elapsed_time(f1), world, dev) / ke
 
+    context = dw5x5_context(wb_arm.sets, K, stream) if world == 1 else None
+
     flops_all = sum_over_ranks(step_flops(wl), world, dev)
     bytes_all = sum_over_ranks(step_bytes(wl), world, dev)
     value = flops_all / (ms_step * 1e-3) / 1e12
@@ -555,6 +587,8 @@ def run_gpu(args, rank, world, local_rank):
     result["e2e"] = {"value": round(flops_all / (e2e_ms * 1e-3) / 1e12, 4), "unit": "TFLOP/s",
                      "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d,
                      "d2h_bytes_per_step": d2h}
+    if context is not None:
+        result["context_dw5x5"] = context
     if clk is not None:
         result["clocks"] = clk
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
