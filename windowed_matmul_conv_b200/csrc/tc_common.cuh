@@ -29,30 +29,8 @@ struct BandTile {
     int nb;
 };
 
-// Calls f(global element offset, byte offset in the slot, bytes) for every
-// contiguous run of the tile (32-bit index math; host checks the ranges).
-template <typename F>
-__device__ __forceinline__ void for_each_band_run(int ws, int W, int H, int C, int nh,
-                                                  const BandTile& t, F&& f)
-{
-    const uint32_t band_bytes = (uint32_t)ws * W * 2;
-    int b = t.band0 / nh;
-    int i = t.band0 - b * nh;
-    int left = t.nb;
-    uint32_t soff = 0;
-    while (left > 0) {
-        const int run = (nh - i) < left ? (nh - i) : left;
-        const long long goff = (((long long)b * C + t.c) * H + (long long)i * ws) * W;
-        f(goff, soff, (uint32_t)run * band_bytes);
-        soff += (uint32_t)run * band_bytes;
-        left -= run;
-        ++b;
-        i = 0;
-    }
-}
-
-// The same runs, addressable one by one so that the lanes of a warp can
-// issue their copies in parallel.  Run 0 starts at band0 and ends at the end
+// The contiguous runs of a tile, addressable one by one so that the lanes of
+// a warp can issue their copies in parallel.  Run 0 starts at band0 and ends at the end
 // of its image plane (or of the tile); every later run is one whole plane or
 // the tile's tail.
 struct BandRuns {
