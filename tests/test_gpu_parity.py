@@ -302,7 +302,12 @@ def test_reparam_merge_argument_errors():
         wb.wbmm_reparam_merge(Tw, Tk, M, 14, 5)       # 5 does not divide 14
     assert e.value.status == 1
     with pytest.raises(wb.WbmmError) as e:
-        wb.wbmm_reparam_merge(Tw, Tk, Tw, 14, 7)      # output overlaps a table
+        wb.wbmm_reparam_merge(Tw, Tk, M, 14, 7)       # a 9x9 table where 7 needs 13x13
+    assert e.value.status == 1
+    Tk7 = gen((2, 13 * 13), 35, scale=0.02)
+    alias = M.view(-1)[:2 * 27 * 27].view(2, 27 * 27)
+    with pytest.raises(wb.WbmmError) as e:
+        wb.wbmm_reparam_merge(alias, Tk7, M, 14, 7)   # output overlaps a table
     assert e.value.status == 1
     assert wb.wbmm_launch_count() == before
 
