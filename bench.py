@@ -385,6 +385,55 @@ def dw5x5_context(sets, K, stream):
     return rec
 
 
+def e2e_pipelined(arm, host_in, host_out, ke, stream):
+    """ms per step of ``ke`` steps through the public API with host buffers,
+    the copies overlapped with the steps: step k runs on buffer set k % 2
+    while the inputs of step k+1 are copied in on one stream and the outputs
+    of step k-1 are copied out on another (host-to-device and device-to-host
+    copies use the link in both directions at once).  Returns None if the
+    streams cannot be set up; the caller then reports the serial figure."""
+    try:
+        sets = arm.sets[:2]
+        cin, cout = torch.cuda.Stream(), torch.cuda.Stream()
+        in_ev = [torch.cuda.Event() for _ in sets]
+        done_ev = [torch.cuda.Event() for _ in sets]
+        out_ev = [torch.cuda.Event() for _ in sets]
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        g0.record(stream)
+        cin.wait_stream(stream)
+        cout.wait_stream(stream)
+        for k in range(ke):
+            j = k % 2
+            s = sets[j]
+            with torch.cuda.stream(cin):
+                cin.wait_event(done_ev[j])        # step k-2 has read this set's inputs
+                for nm, t in host_in.items():
+                    s[nm].copy_(t, non_blocking=True)
+                in_ev[j].record(cin)
+            stream.wait_event(in_ev[j])
+            stream.wait_event(out_ev[j])          # this set's outputs of step k-2 are out
+            if "dT" in host_out:
+                stream.wait_event(out_ev[1 - j])  # dT (one buffer) of step k-1 is out
+            arm.step(j)
+            done_ev[j].record(stream)
+            with torch.cuda.stream(cout):
+                cout.wait_event(done_ev[j])
+                for nm, t in host_out.items():
+                    t.copy_(arm.dT if nm == "dT" else s[nm], non_blocking=True)
+                out_ev[j].record(cout)
+        stream.wait_stream(cout)
+        g1.record(stream)
+        torch.cuda.synchronize()
+        return g0.elapsed_time(g1) / ke
+    except Exception:   # never costs the benchmark line
+        try:
+            torch.cuda.synchronize()
+        except Exception:
+            pass
+        return None
+
+
 def run_gpu(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
@@ -516,6 +565,14 @@ def run_gpu(args, rank, world, local_rank):
     torch.cuda.synchronize()
     barrier(world)
     e2e_ms = max_over_ranks(f0.elapsed_time(f1), world, dev) / ke
+    # the same steps with the copies pipelined: two buffer sets, the next
+    # step's inputs copied in and the previous step's outputs copied out on
+    # their own streams while a step computes
+    barrier(world)
+    pip_ms = e2e_pipelined(wb_arm, host_in, host_out, ke, stream)
+    failed = max_over_ranks(1.0 if pip_ms is None else 0.0, world, dev)   # on any rank
+    pip_ms = None if failed else max_over_ranks(pip_ms, world, dev)
+    barrier(world)
 
     context = dw5x5_context(wb_arm.sets, K, stream) if world == 1 else None
 
@@ -584,9 +641,13 @@ def run_gpu(args, rank, world, local_rank):
     top = alu_tf if wl.dtype == "f32" else peaks["bf16_tflops"]
     step_roof_tf = min(top, step_flops(wl) / step_bytes(wl) * peaks["hbm_gbs"] / 1e3)
     result["step_roofline_frac"] = round(value / world / step_roof_tf, 4)
-    result["e2e"] = {"value": round(flops_all / (e2e_ms * 1e-3) / 1e12, 4), "unit": "TFLOP/s",
-                     "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d,
-                     "d2h_bytes_per_step": d2h}
+    best_ms = pip_ms if pip_ms is not None else e2e_ms
+    result["e2e"] = {"value": round(flops_all / (best_ms * 1e-3) / 1e12, 4), "unit": "TFLOP/s",
+                     "ms_per_step": round(best_ms, 3), "h2d_bytes_per_step": h2d,
+                     "d2h_bytes_per_step": d2h,
+                     "copies": ("overlapped with the steps (2 buffer sets, copy-in and copy-out "
+                                "streams)" if pip_ms is not None else "serial, on the step's stream"),
+                     "ms_per_step_serial": round(e2e_ms, 3)}
     if context is not None:
         result["context_dw5x5"] = context
     if clk is not None:
