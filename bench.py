@@ -355,6 +355,14 @@ def cpu_baseline(wl, host, budget_s=10.0):
                       % (bs, wl.B, wl.C, runs, el)}
 
 
+def workload_label(wl):
+    """The workload's name in both arms' JSON lines."""
+    what = {"train": "forward + dX + dT", "forward": "forward",
+            "cached_dw": "cached forward, then 3x3",
+            "reparam": "cached forward with the merged 14x14 + 7x7 matrix"}[wl.kind]
+    return "%s: B%d C%d %dx%d w%d (%s)" % (wl.name, wl.B, wl.C, wl.H, wl.W, wl.w, what)
+
+
 def dw5x5_context(sets, K, stream):
     """Same-run context, not part of the step: torch's depthwise 5x5
     convolution (padding 2, library kernel) on the step's input maps, the
@@ -593,11 +601,7 @@ def run_gpu(args, rank, world, local_rank):
         "dtype": wl.dtype,
         "data": "synthetic",
         "config": {
-            "workload": "%s: B%d C%d %dx%d w%d (%s)" % (wl.name, wl.B, wl.C, wl.H, wl.W, wl.w,
-                                                      {"train": "forward + dX + dT",
-                                                       "forward": "forward",
-                                                       "cached_dw": "cached forward, then 3x3",
-                                                       "reparam": "cached forward with the merged 14x14 + 7x7 matrix"}[wl.kind]),
+            "workload": workload_label(wl),
             "B": wl.B, "C_per_gpu": wl.C, "H": wl.H, "W": wl.W, "w": wl.w,
             "parallelism": "channel-sharded, %d rank(s), no collective" % world,
             "channels_of_rank0": list(channel_range(wl.C * world, world, 0)),
@@ -699,8 +703,7 @@ def run_reference(args, rank, world):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(el / args.steps * 1e3, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": "%s: B%d C%d %dx%d w%d, sampled" % (wl.name, wl.B, wl.C, wl.H,
-                                                                   wl.W, wl.w)},
+        "config": {"workload": workload_label(wl), "sample": sample},
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s",
                          "cores": oracle.num_threads(), "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
