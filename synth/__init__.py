@@ -12,6 +12,8 @@ Draw recipe (one CPU ``torch.Generator`` seeded once, fixed draw order):
                                         until none is left
   3. dY ~ N(0, 1)                      shape [B, C, H, W]   (training workloads)
   4. K  ~ N(0, 1/9)                    shape [C, 1, 3, 3]   (3x3 mixing weights)
+  5. Tk ~ N(0, 0.02^2)                 shape [C, (2k-1)^2]  (second-branch table of
+                                        the reparameterisation workloads, k = 7)
 All values are drawn in fp32 and then cast (round to nearest even) to the
 workload's dtype; the cast values are the inputs of record.
 """
@@ -33,7 +35,7 @@ class Workload:
     w: int
     dtype: str          # "f32" or "bf16"
     table: str          # "normal" or "truncated"
-    kind: str           # "forward", "train" or "cached_dw"
+    kind: str           # "forward", "train", "cached_dw" or "reparam"
 
     @property
     def d(self):
