@@ -105,7 +105,9 @@ def kernel_bytes(wl, name):
             "backward": 3 * m + tbl + wl.C * wl.t * 4,
             "forward_cached": 2 * m + wl.C * wl.d * wl.d * e,
             "forward_cached_dw3x3": 2 * m + wl.C * wl.d * wl.d * e + wl.C * 9 * e,
-            "reparam_merge": wl.C * wl.d * wl.d * e + tbl,
+            # the merged matrix written, both tables read
+            "reparam_merge": wl.C * wl.d * wl.d * e + tbl
+                             + wl.C * (2 * synth.REPARAM_SMALL_WINDOW - 1) ** 2 * e,
             "dw3x3": 2 * m + wl.C * 9 * e}[name]
 
 
