@@ -132,8 +132,33 @@ def pin_batch_permutation(orc):
     assert np.array_equal(orc.forward(x[perm], T, w), orc.forward(x, T, w)[perm])
 
 
+def _worked_example():
+    path = os.path.join(os.path.dirname(__file__), "golden", "worked_example_w2.txt")
+    g = {}
+    for line in open(path):
+        if line.strip() and not line.startswith("#"):
+            k, *v = line.split()
+            g[k] = np.array([float(t) for t in v])
+    return g
+
+
+def pin_worked_example(orc):
+    # hand-computed values (tests/golden/worked_example_w2.txt) pin the index
+    # convention, the window layout, both gradients, the cached matrix and the
+    # 3x3 mixing to numbers
+    g, w = _worked_example(), 2
+    x, T, dy = g["x"].reshape(1, 1, 2, 4), g["T"].reshape(1, 9), g["dY"].reshape(1, 1, 2, 4)
+    y = orc.forward(x, T, w)
+    assert np.array_equal(y.reshape(-1), g["y"])
+    assert np.array_equal(orc.backward_dx(dy, T, w).reshape(-1), g["dX"])
+    assert np.array_equal(orc.backward_dt(x, dy, w).reshape(-1), g["dT"])
+    assert np.array_equal(orc.expand(T, w).reshape(-1), g["M"])
+    assert np.array_equal(orc.dw3x3(g["y"].reshape(1, 1, 2, 4), g["K"].reshape(1, 1, 3, 3))
+                          .reshape(-1), g["z"])
+
+
 FORWARD_PINS = [pin_identity, pin_shift, pin_constant_table, pin_conv_equivalence,
-                pin_window_locality, pin_batch_permutation]
+                pin_window_locality, pin_batch_permutation, pin_worked_example]
 
 
 # --------------------------------------------------------------------------
@@ -220,7 +245,8 @@ def pin_dt_sum_invariant(orc):
 
 
 GRADIENT_PINS = [pin_dx_adjoint, pin_dx_finite_difference, pin_dt_finite_difference,
-                 pin_dt_adjoint, pin_dt_count_closed_form, pin_dt_sum_invariant]
+                 pin_dt_adjoint, pin_dt_count_closed_form, pin_dt_sum_invariant,
+                 pin_worked_example]
 
 
 # --------------------------------------------------------------------------
@@ -266,8 +292,8 @@ def pin_reparam_merge(orc):
                                    rtol=1e-12, atol=1e-12)
 
 
-OTHER_PINS = [pin_expand, pin_dw3x3, pin_reparam_merge]
-ALL_PINS = FORWARD_PINS + GRADIENT_PINS + OTHER_PINS
+OTHER_PINS = [pin_expand, pin_dw3x3, pin_reparam_merge, pin_worked_example]
+ALL_PINS = list(dict.fromkeys(FORWARD_PINS + GRADIENT_PINS + OTHER_PINS))
 
 
 @pytest.mark.parametrize("pin", ALL_PINS, ids=lambda f: f.__name__)
@@ -391,3 +417,4 @@ def test_planted_mistake_is_caught(mutant):
         orc = _compile_mutant(_mutate(src, func, old, new), td, name)
         caught = _fails_some(pins, orc)
     assert caught is not None, f"no pin caught the planted mistake {name}"
+
