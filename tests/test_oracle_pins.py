@@ -155,6 +155,8 @@ def pin_worked_example(orc):
     assert np.array_equal(orc.expand(T, w).reshape(-1), g["M"])
     assert np.array_equal(orc.dw3x3(g["y"].reshape(1, 1, 2, 4), g["K"].reshape(1, 1, 3, 3))
                           .reshape(-1), g["z"])
+    assert np.array_equal(orc.reparam_merge(T, g["Tk"].reshape(1, 1), w, 1).reshape(-1),
+                          g["Mmerged"])
 
 
 FORWARD_PINS = [pin_identity, pin_shift, pin_constant_table, pin_conv_equivalence,
