@@ -15,7 +15,8 @@
  *     the window, inter-block 3x3 depthwise mixing, inference caching);
  *   - the arxivdaily.com English abstract (contiguous windows, compact
  *     relative position bias table, batched matrix multiplication).
- * The pages print no formula.  The index convention fixed for this build is
+ * The pages print no formula.  The index convention used here (offset =
+ * output minus input position, row-major over the two offsets) is
  *   M_c[(p,q),(r,s)] = T_c[(p-r+w-1)(2w-1) + (q-s+w-1)],
  * with (p,q) the output and (r,s) the input position inside one window.
  *
