@@ -32,7 +32,6 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 import synth  # noqa: E402
-from windowed_matmul_conv_b200.sharding import channel_range  # noqa: E402
 
 METRIC = "WBMM fwd/bwd TFLOP/s, HBM GB/s and % of roofline at w=14 bf16 on 1 B200"
 L2_BYTES = 126 * 2 ** 20
@@ -210,7 +209,8 @@ class Arm:
         if wl.kind == "train":
             self.dT = torch.empty((wl.C, wl.t), dtype=torch.float32, device=dev)
             nbytes = wb.wbmm_backward_workspace_bytes(wl.B, wl.C, wl.H, wl.W, wl.w, torch.bfloat16)
-            self.ws = torch.empty(max(1, nbytes // 4), dtype=torch.float32, device=dev)
+            # zero-filled once: the table gradient's arrival counters start at zero
+            self.ws = torch.zeros(max(1, nbytes // 4), dtype=torch.float32, device=dev)
         if wl.kind == "reparam":
             self.Tk = d["Tk"].to(dev)
             self.M = wb.reparam_merge(self.T, self.Tk, wl.w, synth.REPARAM_SMALL_WINDOW)
@@ -444,11 +444,119 @@ def e2e_pipelined(arm, host_in, host_out, ke, stream):
         return None
 
 
+class GraphSteps:
+    """CUDA graphs of an arm's steps: one holding a step on each buffer set in
+    turn (the kernels of consecutive steps overlap their prologues and tails
+    through programmatic dependent launch, as in a training loop) and one
+    single step per set for the remainder of K."""
+
+    def __init__(self, arm):
+        self.nsets = len(arm.sets)
+        self.all = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.all):
+            for k in range(self.nsets):
+                arm.step(k)
+        self.one = []
+        for k in range(self.nsets):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                arm.step(k)
+            self.one.append(g)
+        self.all.replay()
+        for g in self.one:
+            g.replay()
+        torch.cuda.synchronize()
+
+    def replay(self, K):
+        full, rest = divmod(K, self.nsets)
+        for _ in range(full):
+            self.all.replay()
+        for k in range(rest):
+            self.one[k].replay()
+
+    def release(self):
+        del self.all
+        self.one = []
+
+
+def roofline_of(wl, value_tf, peaks):
+    """Fraction of the step's roofline, min(tensor peak, AI x HBM), that the
+    step's algorithmic throughput reaches (burst tensor peak; fp32 steps
+    against the CUDA-core FMA peak)."""
+    top = peaks["bf16_tflops"] if wl.dtype == "bf16" else peaks["fp32_fma_tflops"]
+    ai = step_flops(wl) / step_bytes(wl)
+    roof = min(top, ai * peaks["hbm_gbs"] / 1e3)
+    return {"bound": "tensor" if roof >= top else "hbm", "roofline_tflops": round(roof, 1),
+            "frac": round(value_tf / roof, 4)}
+
+
+# The benchmark's other workloads, timed after the headline step on one GPU
+WORKLOAD_SWEEP = ("fwd", "sweep7", "sweep14", "sweep28", "cached")
+
+
+def time_workloads(dev, peaks, K):
+    """Graph-timed device time of every other workload (K steps each after 3
+    warm-up steps, 3 rotating buffer sets larger than L2), with the fused
+    cached forward + 3x3 timed beside its two-call step.  Never raises: a
+    failing workload is reported in its record."""
+    out = {}
+    for key in WORKLOAD_SWEEP:
+        wl = synth.WORKLOADS[WORKLOADS[key]]
+        rec = {"workload": workload_label(wl)}
+        try:
+            arm = Arm(wl, seed=0, nsets=3, dev=dev)
+            for k in range(3):
+                arm.step(k)
+            torch.cuda.synchronize()
+            gs = GraphSteps(arm)
+            stream = torch.cuda.current_stream()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            prefill(5.0)
+            e0.record(stream)
+            gs.replay(K)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            gs.release()
+            ms = e0.elapsed_time(e1) / K
+            tf = step_flops(wl) / (ms * 1e-3) / 1e12
+            rec.update({"us": round(ms * 1e3, 2), "tflops": round(tf, 1),
+                        "gbs": round(step_bytes(wl) / (ms * 1e-3) / 1e9, 1),
+                        "windows_channels_per_s": round(wl.windows_per_channel * wl.C
+                                                        / (ms * 1e-3), 1),
+                        "calls": arm.calls()})
+            rec.update(roofline_of(wl, tf, peaks))
+            for name in arm.alternatives():
+                s = arm.sets[0]
+                for _ in range(3):
+                    arm.launch(name, s)
+                a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                torch.cuda.synchronize()
+                a0.record(stream)
+                for k in range(K):
+                    arm.launch(name, arm.sets[k % len(arm.sets)])
+                a1.record(stream)
+                torch.cuda.synchronize()
+                us = a0.elapsed_time(a1) / K * 1e3
+                rec.setdefault("alternatives", {})[name] = {
+                    "us": round(us, 2), "gbs": round(kernel_bytes(wl, name) / (us * 1e-6) / 1e9, 1),
+                    "frac_of_step_roofline": round(step_flops(wl) / (us * 1e-6) / 1e12
+                                                   / rec["roofline_tflops"], 4)}
+            assert arm.wb.wbmm_get_device_status() == 0, "device status"
+            del arm
+        except Exception as e:   # reported, never costs the headline line
+            rec["error"] = ("%s: %s" % (type(e).__name__, e))[:200]
+        torch.cuda.empty_cache()
+        out[key] = rec
+    return out
+
+
 def run_gpu(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     wl = synth.WORKLOADS[WORKLOADS[args.workload]]
+    from windowed_matmul_conv_b200.sharding import channel_range
     peaks = load_peaks()
+    peaks["fp32_fma_tflops"] = fp32_fma_peak_tflops(dev)
     wb_arm = Arm(wl, seed=rank, nsets=3, dev=dev)
     wb = wb_arm.wb
     K, W = args.steps, args.warmup
@@ -460,25 +568,7 @@ def run_gpu(args, rank, world, local_rank):
     torch.cuda.synchronize()
     assert wb.wbmm_get_device_status() == 0, "device status after warm-up"
 
-    # CUDA graphs: one holding a step on each buffer set in turn (the
-    # kernels of consecutive steps overlap their prologues and tails through
-    # programmatic dependent launch, as in a training loop), and one single
-    # step per set for the remainder of K
-    nsets = len(wb_arm.sets)
-    graph_all = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph_all):
-        for k in range(nsets):
-            wb_arm.step(k)
-    graphs = []
-    for k in range(nsets):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            wb_arm.step(k)
-        graphs.append(g)
-    graph_all.replay()
-    for g in graphs:
-        g.replay()
-    torch.cuda.synchronize()
+    gsteps = GraphSteps(wb_arm)
 
     clocks = ClockSampler(local_rank)
     clocks.start()
@@ -491,11 +581,7 @@ def run_gpu(args, rank, world, local_rank):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     prefill()
     e0.record(stream)
-    full, rest = divmod(K, nsets)
-    for _ in range(full):
-        graph_all.replay()
-    for k in range(rest):
-        graphs[k].replay()
+    gsteps.replay(K)
     e1.record(stream)
     torch.cuda.synchronize()
     barrier(world)
@@ -660,9 +746,17 @@ def run_gpu(args, rank, world, local_rank):
         result["clocks"] = clk
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(wl, wb_arm.host)
-    del graph_all
-    for g in graphs:
-        del g
+    gsteps.release()
+    if world == 1 and not args.no_workloads:
+        # the other workloads, each in its own graphs, with a clock record
+        wclk = ClockSampler(local_rank)
+        wclk.start()
+        time.sleep(0.3)
+        recs = time_workloads(dev, peaks, max(5, min(K, 20)))
+        c = wclk.stop()
+        result["workloads"] = {"steps_each": max(5, min(K, 20)), "records": recs}
+        if c is not None:
+            result["workloads"]["clocks"] = c
     return result
 
 
@@ -713,6 +807,19 @@ def run_reference(args, rank, world):
     }
 
 
+def spawn_ranks(n):
+    """Starts one process per GPU (torch.distributed.run on this node, the
+    rendezvous on 127.0.0.1) with the same arguments; returns its exit code."""
+    import socket
+    with socket.socket() as so:
+        so.bind(("127.0.0.1", 0))
+        port = so.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           "--nproc-per-node", str(n), "--master-addr", "127.0.0.1",
+           "--master-port", str(port), os.path.abspath(__file__)] + sys.argv[1:]
+    return subprocess.call(cmd)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -721,11 +828,22 @@ def main():
     ap.add_argument("--impl", choices=["wbmm", "reference"], default="wbmm")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="train")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the other workloads' timings after the headline step")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "wbmm":
         ap.error("at least 3 warm-up steps")
+    if args.gpus < 1:
+        ap.error("--gpus must be at least 1")
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
+    env_world = os.environ.get("WORLD_SIZE")
+    if env_world is None and args.gpus > 1:
+        sys.exit(spawn_ranks(args.gpus))
+    world = int(env_world or "1")
+    if world != args.gpus:
+        ap.error("--gpus %d but WORLD_SIZE=%d: launch one process per GPU "
+                 "(torchrun --nproc-per-node %d), or omit WORLD_SIZE and let "
+                 "bench.py start the ranks" % (args.gpus, world, args.gpus))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":

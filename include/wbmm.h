@@ -80,10 +80,19 @@ WBMM_API wbmm_status wbmm_forward(const void *x, const void *T, void *y,
                          wbmm_dtype dt, void *stream);
 
 /*
- * Bytes of device workspace wbmm_backward needs for the table gradient:
- * fp32 partial tables, one per (channel, fixed chunk of windows).  The chunk
- * split depends only on the shape, the device's SM count and whether dX is
- * computed in the same call, so dT is bit-identical from run to run.
+ * Bytes of device workspace wbmm_backward needs for the table gradient.
+ * bf16 on the tensor-core kernels: fp32 partial tables of the channels whose
+ * windows are split between CTAs, then one 32-bit arrival counter per channel
+ * (the workspace's last C 32-bit words).  Zero-fill the workspace once before
+ * its first use (cudaMemset, torch.zeros); every call leaves the counters at
+ * zero again, a call that ends in WBMM_ERR_TIMEOUT included, so the same
+ * workspace serves any number of later calls, graph replays included.  A
+ * call that ends in WBMM_ERR_CUDA may leave it dirty: zero it again.
+ * fp32 (and bf16 shapes outside the tensor-core kernels): fp32 partial tables,
+ * one per (channel, fixed chunk of windows); prior content does not matter.
+ * The split depends only on the shape, the device's SM count and whether dX
+ * is computed in the same call, so dT is bit-identical from run to run.
+ * Calls that share a workspace must not overlap on the GPU.
  * Returns 0 for invalid shapes.
  */
 WBMM_API size_t wbmm_backward_workspace_bytes(int B, int C, int H, int W, int w, wbmm_dtype dt);
@@ -180,8 +189,11 @@ WBMM_API wbmm_status wbmm_dw3x3(const void *y, const void *K, void *z,
  * the array's device address (cudaGetSymbolAddress); make that first call
  * before any stream capture.  Every device holds the array until exit.  All
  * calls share it, so calls whose work overlaps on the GPU race and must be
- * ordered by the caller.  Returns WBMM_ERR_WORKSPACE when C times the number
- * of partial tables times (2w-1)^2 exceeds 2^20 floats.
+ * ordered by the caller.  The array starts zeroed and every call leaves its
+ * arrival counters at zero (see wbmm_backward_workspace_bytes).  Returns
+ * WBMM_ERR_WORKSPACE, before any launch, when the workspace that
+ * wbmm_backward_workspace_bytes reports for the same shape and a dT-only call
+ * exceeds the array's 2^20 floats (4 MiB).
  */
 WBMM_API wbmm_status wbmm_backward_dt_static(const void *x, const void *dY, float *dT,
                                              int B, int C, int H, int W, int w,

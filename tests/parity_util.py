@@ -6,8 +6,12 @@ bf16 path (fp32 accumulation, bf16 output):
     the forward); bf16 output rounding alone is at most 2^-9 of it;
   * whole tensor sum|gpu - ref| / sum|ref| <= 5e-3 (mean relative error as an
     L1 ratio, which stays finite where single outputs are near zero).
-fp32 path: per element |gpu - ref| / sum_v |M_uv x_v| <= 1e-5; fp32
-accumulation of d terms is bounded by d * 2^-24 of that sum (2.9e-6 at d=49).
+fp32 path: the gate is componentwise for every element,
+|gpu - ref| <= 1e-5 * sum_v |M_uv x_v| (the magnitude of the output's terms,
+which is never below |ref|); fp32 accumulation of d terms is bounded by
+d * 2^-24 of that sum (2.9e-6 at d=49).  Beside it the check reports the plain
+relative error |gpu - ref| / |ref| over the outputs with |ref| at least 1e-2
+of their terms' magnitude, where it is meaningful.
 """
 import numpy as np
 
@@ -53,10 +57,18 @@ def check_bf16(gpu, ref, bound, what):
 
 
 def check_f32(gpu, ref, absdot, what):
-    rel = np.abs(gpu - ref) / np.maximum(np.maximum(np.abs(ref), absdot), 1e-300)
-    worst = float(rel.max())
-    assert worst <= F32_REL_TOL, f"{what}: max relative error {worst:.3e}"
-    return worst
+    """Gate: componentwise error <= F32_REL_TOL of the terms' magnitude.
+    Returns (worst componentwise error, worst plain relative error over the
+    outputs with |ref| >= 1e-2 * absdot, or 0.0 if there are none)."""
+    err = np.abs(gpu - ref)
+    comp = err / np.maximum(np.maximum(np.abs(ref), absdot), 1e-300)
+    worst = float(comp.max())
+    big = np.abs(ref) >= 1e-2 * absdot
+    plain = float((err[big] / np.abs(ref[big])).max()) if big.any() else 0.0
+    print("%s: componentwise %.3e, plain relative (|ref| >= 1e-2 of terms) %.3e"
+          % (what, worst, plain))
+    assert worst <= F32_REL_TOL, f"{what}: max componentwise error {worst:.3e}"
+    return worst, plain
 
 
 def dt_bound(x, dy, w):

@@ -68,19 +68,20 @@ def test_workspace_size_formula(lib):
     f.restype = ctypes.c_size_t
     f.argtypes = [ctypes.c_int] * 6
     # bf16, tensor-core path: one partial table per (channel, CTA range)
-    # segment, at most n = C + min(256, tiles) - 1 of them, then one 64-bit
-    # flag per table (8-byte aligned).
-    def tc(n, tsz=729):
-        return ((n * tsz + 1) // 2 * 2 + 2 * n) * 4
+    # segment, at most n = C + min(256, tiles) - 1 of them, then one 32-bit
+    # arrival counter per channel (16-byte aligned).
+    def tc(C, grid, tsz=729):
+        n = C + grid - 1
+        return ((n * tsz + 3) // 4 * 4 + C) * 4
     # training workload: 64-window tiles of 32 two-window bands, 8 tiles per
     # channel, 2048 tiles -> 256 + 255 tables
-    assert f(128, 256, 28, 28, 14, 1) == tc(256 + 255)
+    assert f(128, 256, 28, 28, 14, 1) == tc(256, 256)
     # 64 images of 56x56: 16 bands/tile, 16 tiles/channel, 2048 tiles
-    assert f(64, 128, 56, 56, 14, 1) == tc(128 + 255)
+    assert f(64, 128, 56, 56, 14, 1) == tc(128, 256)
     # 32 images of 112x112: 8 bands/tile, 32 tiles/channel, 128 tiles
-    assert f(32, 4, 112, 112, 14, 1) == tc(4 + 127)
+    assert f(32, 4, 112, 112, 14, 1) == tc(4, 128)
     # 2 images of 112x112, w = 7: 64-window tiles of 4 bands, 8 tiles/channel
-    assert f(2, 4, 112, 112, 7, 1) == tc(4 + 31, 169)
+    assert f(2, 4, 112, 112, 7, 1) == tc(4, 32, 169)
     # fp32, CUDA-core path: chunks of 8 bands per channel
     assert f(2, 3, 14, 28, 7, 0) == 3 * 1 * 169 * 4
     assert f(1, 1, 14, 15, 7, 1) == 0

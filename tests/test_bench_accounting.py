@@ -80,3 +80,35 @@ def test_merge_counts(bench):
     # 96 merged 196 x 196 matrices written, a 27^2 and a 13^2 table read
     assert bench.kernel_bytes(wl, "reparam_merge") == 96 * (196 * 196 + 729 + 169) * 2
     assert bench.step_bytes(wl) == 2 * 8 * 96 * 224 * 224 * 2 + 96 * 196 * 196 * 2
+
+
+def _run_bench(args, env_extra, code_tail=""):
+    import subprocess
+    env = dict(os.environ)
+    env.pop("WORLD_SIZE", None)
+    env.update(env_extra)
+    code = ("import sys, runpy; sys.argv = ['bench.py'] + %r\n"
+            "try:\n    runpy.run_path('bench.py', run_name='__main__')\n"
+            "except SystemExit as e:\n    print('EXIT', e.code)\n%s" % (list(args), code_tail))
+    return subprocess.run([sys.executable, "-c", code], cwd=ROOT, env=env, capture_output=True,
+                          text=True, timeout=600)
+
+
+def test_gpus_flag_must_match_the_launched_ranks():
+    # one process launched (WORLD_SIZE=1) but --gpus 2 asked: refused loudly,
+    # before any device work, instead of timing one GPU as if it were two
+    r = _run_bench(["--gpus", "2", "--steps", "3", "--warmup", "3"], {"WORLD_SIZE": "1"})
+    assert "EXIT 2" in r.stdout
+    assert "--gpus 2 but WORLD_SIZE=1" in r.stderr
+
+
+def test_reference_arm_maps_no_wbmm_library():
+    # the oracle arm runs the CPU oracle only: the CUDA library is never loaded
+    tail = ("maps = open('/proc/self/maps').read()\n"
+            "print('LIBWBMM' if 'libwbmm' in maps else 'CLEAN')\n"
+            "print('ORACLE' if 'liboracle' in maps else 'NO-ORACLE')\n")
+    r = _run_bench(["--impl", "reference", "--workload", "fwd", "--steps", "1", "--warmup", "0"],
+                   {}, tail)
+    assert r.returncode == 0, r.stderr
+    assert '"impl": "reference"' in r.stdout
+    assert "CLEAN" in r.stdout and "ORACLE" in r.stdout

@@ -4,9 +4,11 @@ Hosts with a fixed device-memory budget, plugins inside frameworks that own
 every device allocation, and paths where cudaMalloc would synchronise the
 device cannot hand wbmm_backward a workspace.  This entry point keeps the
 partial tables in a fixed array inside the library instead.  The test calls
-it through the C ABI twice in a row per shape and checks each result against
-wbmm_backward's dT: bit-identical (same kernels, same partial split) and, as
-for every parity test, within the bf16/fp32 tolerances against its bound.
+it through the C ABI twice in a row per shape, with new inputs for the
+second call, and checks each result against the fp64 oracle within the
+bf16/fp32 tolerances of every parity test, and against wbmm_backward's dT
+on the same inputs, which it must equal bit for bit (same kernels, same
+partial split).
 This file sorts last so a run that stops at the first failure has already
 run every other test; it also passes alone in a fresh process.
 """
@@ -33,24 +35,25 @@ SHAPES = [
 
 
 @pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "x".join(map(str, s[:5])) + str(s[5])[-4:])
-def test_static_scratch_matches_workspace_path(shape):
+def test_static_scratch_matches_oracle_and_workspace_path(shape):
     B, C, H, W, w, dtype = shape
-    x = synth.draw_tensor((B, C, H, W), 41, "f32").to(dtype).cuda()
-    dy = synth.draw_tensor((B, C, H, W), 42, "f32").to(dtype).cuda()
-    _, ref = wb.backward(x, None, dy, w, need_dx=False)
-    torch.cuda.synchronize()
-    xr, gr = to_np(x), to_np(dy)
-    for _ in range(2):
+    for call in range(2):
+        x = synth.draw_tensor((B, C, H, W), 41 + 2 * call, "f32").to(dtype).cuda()
+        dy = synth.draw_tensor((B, C, H, W), 42 + 2 * call, "f32").to(dtype).cuda()
         dT = torch.full((C, (2 * w - 1) ** 2), float("nan"), dtype=torch.float32, device="cuda")
         wb.wbmm_backward_dt_static(x, dy, dT, w)
         torch.cuda.synchronize()
         assert wb.wbmm_get_device_status() == 0
-        assert torch.equal(dT, ref)
+        xr, gr = to_np(x), to_np(dy)
+        ref = oracle.backward_dt(xr, gr, w)
         if dtype == torch.bfloat16:
-            check_bf16(to_np(dT), to_np(ref), dt_bound(xr, gr, w), "static dT vs workspace dT")
+            check_bf16(to_np(dT), ref, dt_bound(xr, gr, w), "static dT, call %d" % call)
         else:
             absdt = oracle.backward_dt(np.abs(xr), np.abs(gr), w)
-            check_f32(to_np(dT), to_np(ref), absdt, "static dT vs workspace dT")
+            check_f32(to_np(dT), ref, absdt, "static dT, call %d" % call)
+        _, ws_dT = wb.backward(x, None, dy, w, need_dx=False)
+        torch.cuda.synchronize()
+        assert torch.equal(dT, ws_dT)
 
 
 def test_static_scratch_rejects_oversized_calls():

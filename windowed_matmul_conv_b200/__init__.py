@@ -239,7 +239,8 @@ def backward(x, T, dY, w, need_dx=True, need_dt=True, stream=None):
     ws = None
     if need_dt:
         nbytes = wbmm_backward_workspace_bytes(B, C, H, W, w, dY.dtype)
-        ws = torch.empty(max(1, nbytes // 4), dtype=torch.float32, device=dY.device)
+        # zero-filled: the table gradient's arrival counters start at zero
+        ws = torch.zeros(max(1, nbytes // 4), dtype=torch.float32, device=dY.device)
     wbmm_backward(x, T, dY, dX, dT, ws, w, stream)
     return dX, dT
 

@@ -105,39 +105,19 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t *bar, uint32_t parity,
     return true;
 }
 
-// ------------------------------------------------ flags between CTAs
-__device__ __forceinline__ void st_release_u64(unsigned long long *p, unsigned long long v)
+// ------------------------------------------------ counters between CTAs
+// Device-scope atomic add with acquire-release order: the caller's earlier
+// writes (made visible to it by a fence and a barrier of its CTA) are
+// released with the increment, and the writes released by every earlier
+// increment of the same word are acquired.  Returns the old value.
+__device__ __forceinline__ unsigned int atom_add_acq_rel_u32(unsigned int *p, unsigned int v)
 {
-    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-}
-
-__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long *p)
-{
-    unsigned long long v;
-    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-    return v;
-}
-
-// Bounded wait until *p == token (written by another CTA of the same grid).
-// Gives up on the abort flag or after `budget` SM cycles; in the second case
-// it raises the abort flag and the device status word.  Returns true when the
-// token arrived.
-__device__ __forceinline__ bool wait_token(const unsigned long long *p, unsigned long long token,
-                                           volatile int *abort, unsigned long long budget,
-                                           int *status)
-{
-    const long long t0 = clock64();
-    while (ld_acquire_u64(p) != token) {
-        if (*abort)
-            return false;
-        if ((unsigned long long)(clock64() - t0) > budget) {
-            *abort = 1;
-            atomicOr(status, kStatusTimeout);
-            return false;
-        }
-        __nanosleep(256);
-    }
-    return true;
+    unsigned int old;
+    asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], %2;"
+                 : "=r"(old)
+                 : "l"(p), "r"(v)
+                 : "memory");
+    return old;
 }
 
 // ------------------------------------------------------- 4-byte async copies

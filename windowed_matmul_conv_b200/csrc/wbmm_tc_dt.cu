@@ -8,18 +8,24 @@
 //
 // The channels' tiles, in channel order, are split into one contiguous,
 // balanced range per CTA: of whole channels when that gives no CTA more tiles
-// than a split at tile granularity, else of tiles.  A segment is the part of a CTA's range inside one
-// channel; each segment ends with one reduction of G into its own fp32 partial
-// table, at index c + k (channel c, CTA k: ranges are ordered, so the index
-// is unique).  A channel inside one CTA's range is written to dT directly.
-// A channel split between CTAs k0 < ... < k1 is the last segment of CTA k0
-// and an earlier segment of every later one: those write their partial table
-// and then a flag word holding this launch's 64-bit token (release); k0 waits
-// for the flags (bounded) and adds its own sums and then the later partials,
-// in CTA order, into dT.  Stale flags hold other launches' tokens, so the
-// workspace needs no initialisation.  Every sum runs in a fixed order, so the
-// result is bit-identical from run to run for a given grid (the device's SM
-// count).
+// than a split at tile granularity, else of tiles.  A segment is the part of a
+// CTA's range inside one channel; each segment ends with one reduction of G
+// into its own fp32 partial table.  A channel inside one CTA's range is
+// written to dT directly.  A channel split between CTAs k0 < ... < k1 is
+// finished by whichever of them arrives last: each writes its segment's
+// partial table (at index c + k of the workspace: ranges are ordered, so the
+// index is unique) and then adds one to the channel's arrival counter
+// (acquire-release, device scope); the CTA that sees the count reach
+// k1 - k0 + 1 adds the partial tables in CTA order k0, ..., k1 into dT and
+// sets the counter back to zero.  No CTA ever waits for another, so the grid
+// need not be co-resident, and a counter can only reach its final count
+// within one launch: a re-launch with the same arguments (a replayed graph)
+// never sees the previous launch's partials as ready.  Every counter starts
+// at zero (the workspace's counter words must be zero before the first call)
+// and every launch leaves it zero, the aborted ones included, since each CTA
+// arrives once per split channel whether or not its waits succeeded.  Every
+// sum runs in a fixed order, so the result is bit-identical from run to run
+// for a given grid (the device's SM count).
 //
 // Per tile the producer bulk-copies the dY and x bands into a raw slot; the
 // transform warps write both tiles in the layout of the forward kernel's
@@ -35,9 +41,6 @@
 // (fixed p order) into registers.  The last half's sums are the segment's
 // partial table.
 #include <cuda_bf16.h>
-
-#include <atomic>
-#include <chrono>
 
 #include "ptx_sm100.cuh"
 #include "tc_common.cuh"
@@ -99,8 +102,7 @@ struct TcDtParams {
     const uint16_t* x;
     const uint16_t* dy;
     float* partials;        // [C + grid - 1][tsz], segment (c, k) at c + k
-    unsigned long long* flags;  // [C + grid - 1], token when partial c + k is written
-    unsigned long long token;   // unique per launch
+    unsigned int* counters; // [C] segments of channel c written so far (zero between launches)
     float* dT;              // [C][tsz]
     int C, H, W, nh, nw;
     int bpt;
@@ -130,8 +132,7 @@ struct DtBars {
     uint64_t fin;
     uint32_t tmem_slot;
     int abort;
-    int seg_ok;             // the later segments of the current channel arrived
-    int pre_ok;             // ... and did so before its reduction began
+    int last;               // this CTA is the last to arrive at the current split channel
 };
 
 struct DtTile {
@@ -396,37 +397,6 @@ __global__ void __launch_bounds__(kDtThreads, 1) wbmm_tc_dt_kernel(const __grid_
             const int k = (int)blockIdx.x;
             const int k0 = dt_cta_of(P, (long long)c * P.tpc);
             const int k1 = dt_cta_of(P, (long long)c * P.tpc + P.tpc - 1);
-            // The channel's first tiles and last segment: the later segments
-            // (one or two CTAs) were normally published long ago, so their
-            // partial sums are fetched now and arrive during the reduction.
-            const bool gather = k == k0 && k1 > k0 && k1 - k0 <= 2;
-            float pre[2][NBT];
-            bool pre_ok = false;
-            if (gather) {
-                if (et == 0) {
-                    int r = 1;
-                    for (int kk = k0 + 1; kk <= k1; ++kk)
-                        r &= ld_acquire_u64(P.flags + c + kk) == P.token ? 1 : 0;
-                    S.pre_ok = r;
-                }
-                named_bar_sync(3, kDtEpiThreads);
-                pre_ok = S.pre_ok != 0;
-                named_bar_sync(3, kDtEpiThreads);   // pre_ok is rewritten next
-                if (pre_ok && ok) {
-                    __threadfence();
-#pragma unroll
-                    for (int j = 0; j < 2; ++j) {
-#pragma unroll
-                        for (int i = 0; i < NBT; ++i) {
-                            const int bin = et + i * kDtEpiThreads;
-                            pre[j][i] = (k0 + 1 + j <= k1 && bin < F::TSZ)
-                                            ? __ldcg(P.partials +
-                                                     (long long)(c + k0 + 1 + j) * F::TSZ + bin)
-                                            : 0.0f;
-                        }
-                    }
-                }
-            }
             float acc[NBT];
 #pragma unroll
             for (int i = 0; i < NBT; ++i)
@@ -514,8 +484,9 @@ __global__ void __launch_bounds__(kDtThreads, 1) wbmm_tc_dt_kernel(const __grid_
                 }
                 continue;
             }
-            if (k != k0) {
-                // an earlier segment of this CTA: publish it for CTA k0
+            // a channel split between CTAs: publish this segment's partial
+            // table, then count it; the last CTA to arrive adds all of them
+            {
                 float* out = P.partials + (long long)(c + k) * F::TSZ;
 #pragma unroll
                 for (int i = 0; i < NBT; ++i) {
@@ -523,52 +494,32 @@ __global__ void __launch_bounds__(kDtThreads, 1) wbmm_tc_dt_kernel(const __grid_
                     if (bin < F::TSZ)
                         out[bin] = acc[i];
                 }
-                __threadfence();
-                named_bar_sync(3, kDtEpiThreads);
-                if (et == 0)
-                    st_release_u64(P.flags + c + k, P.token);
-                continue;
             }
-            // this CTA holds the channel's first tiles and its last segment:
-            // add the later segments in CTA order
-            if (pre_ok) {
-                if (ok) {
-#pragma unroll
-                    for (int i = 0; i < NBT; ++i) {
-                        const int bin = et + i * kDtEpiThreads;
-                        if (bin < F::TSZ) {
-                            float sum = acc[i] + pre[0][i];
-                            if (k1 - k0 == 2)
-                                sum += pre[1][i];
-                            P.dT[(long long)c * F::TSZ + bin] = sum;
-                        }
-                    }
-                }
-                continue;
-            }
-            // otherwise wait for them first
+            __threadfence();
+            named_bar_sync(3, kDtEpiThreads);
             if (et == 0) {
-                int good = 1;
-                for (int kk = k0 + 1; kk <= k1 && good; ++kk)
-                    good = wait_token(P.flags + c + kk, P.token, abort, P.budget, P.status);
-                S.seg_ok = good;
+                const unsigned int prev = atom_add_acq_rel_u32(P.counters + c, 1u);
+                const int last = prev == (unsigned int)(k1 - k0);
+                if (last)
+                    atomicExch(P.counters + c, 0u);   // zero again for the next launch
+                S.last = last;
             }
             named_bar_sync(3, kDtEpiThreads);
-            if (ok && S.seg_ok) {
+            if (S.last && ok) {
                 __threadfence();
 #pragma unroll
                 for (int i = 0; i < NBT; ++i) {
                     const int bin = et + i * kDtEpiThreads;
                     if (bin < F::TSZ) {
                         const float* pc = P.partials + (long long)c * F::TSZ + bin;
-                        float sum = acc[i];
+                        float sum = k0 == k ? acc[i] : __ldcg(pc + (long long)k0 * F::TSZ);
                         for (int kk = k0 + 1; kk <= k1; ++kk)
-                            sum += __ldcg(pc + (long long)kk * F::TSZ);
+                            sum += kk == k ? acc[i] : __ldcg(pc + (long long)kk * F::TSZ);
                         P.dT[(long long)c * F::TSZ + bin] = sum;
                     }
                 }
             }
-            named_bar_sync(3, kDtEpiThreads);   // seg_ok is rewritten next
+            named_bar_sync(3, kDtEpiThreads);   // S.last is rewritten next
         }
     }
 
@@ -633,27 +584,11 @@ constexpr int kDtMaxGrid = 256;
 
 long long tc_dt_partials_impl(const Geom& g);
 
-// Float offset of the flag words in the workspace (after the partial tables,
-// rounded up to 8 bytes).
-long long dt_flags_offset(const Geom& g)
+// Float offset of the arrival counters in the workspace (after the partial
+// tables, rounded up to 16 bytes).
+long long dt_counters_offset(const Geom& g)
 {
-    return (tc_dt_partials_impl(g) * g.tsz + 1) / 2 * 2;
-}
-
-// A token no earlier launch of this process used; the start is drawn from
-// the clock and the address space so that another process's stale flags
-// match with probability ~2^-64.
-unsigned long long next_launch_token()
-{
-    static std::atomic<unsigned long long> ctr{0};
-    static const unsigned long long seed = [] {
-        unsigned long long v = (unsigned long long)std::chrono::steady_clock::now()
-                                   .time_since_epoch()
-                                   .count();
-        v ^= (unsigned long long)reinterpret_cast<uintptr_t>(&ctr) * 0x9E3779B97F4A7C15ull;
-        return v | 1ull;
-    }();
-    return seed + 0x9E3779B97F4A7C15ull * (ctr.fetch_add(1) + 1);
+    return (tc_dt_partials_impl(g) * g.tsz + 3) / 4 * 4;
 }
 
 int dt_tiles_per_channel(const Geom& g)
@@ -691,8 +626,7 @@ cudaError_t dt_launch_ws(const Geom& g, const void* x, const void* dy, float* wo
     P.x = static_cast<const uint16_t*>(x);
     P.dy = static_cast<const uint16_t*>(dy);
     P.partials = workspace;
-    P.flags = reinterpret_cast<unsigned long long*>(workspace + dt_flags_offset(g));
-    P.token = next_launch_token();
+    P.counters = reinterpret_cast<unsigned int*>(workspace + dt_counters_offset(g));
     P.dT = dT;
     P.C = g.C; P.H = g.H; P.W = g.W; P.nh = g.nh; P.nw = g.nw;
     P.bpt = F::NT / g.nw;
@@ -768,8 +702,9 @@ long long tc_dt_tiles(const Geom& g)
 
 long long tc_dt_workspace_floats(const Geom& g)
 {
-    // partial tables, then one 64-bit flag per table (8-byte aligned)
-    return dt_flags_offset(g) + 2 * tc_dt_partials(g);
+    // partial tables, then one 32-bit arrival counter per channel (16-byte
+    // aligned), the workspace's last C words
+    return dt_counters_offset(g) + g.C;
 }
 
 cudaError_t tc_dt_launch(const Geom& g, const void* x, const void* dy, float* partials, float* dT,
