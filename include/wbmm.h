@@ -80,16 +80,26 @@ WBMM_API wbmm_status wbmm_forward(const void *x, const void *T, void *y,
                          wbmm_dtype dt, void *stream);
 
 /*
+ * Size of the arrival-counter region at the start of a table-gradient
+ * workspace, in 32-bit words (see wbmm_backward_workspace_bytes).
+ */
+#define WBMM_DT_COUNTER_WORDS 65536
+
+/*
  * Bytes of device workspace wbmm_backward needs for the table gradient.
- * bf16 on the tensor-core kernels: fp32 partial tables of the channels whose
- * windows are split between CTAs, then one 32-bit arrival counter per channel
- * (the workspace's last C 32-bit words).  Zero-fill the workspace once before
- * its first use (cudaMemset, torch.zeros); every call leaves the counters at
- * zero again, a call that ends in WBMM_ERR_TIMEOUT included, so the same
- * workspace serves any number of later calls, graph replays included.  A
- * call that ends in WBMM_ERR_CUDA may leave it dirty: zero it again.
- * fp32 (and bf16 shapes outside the tensor-core kernels): fp32 partial tables,
- * one per (channel, fixed chunk of windows); prior content does not matter.
+ * bf16 on the tensor-core kernels (C <= WBMM_DT_COUNTER_WORDS): the workspace
+ * starts with WBMM_DT_COUNTER_WORDS 32-bit arrival counters (256 KiB; word c
+ * counts the CTAs that have finished their part of channel c), followed by
+ * fp32 partial tables of the channels whose windows are split between CTAs.
+ * Zero-fill the workspace once before its first use (cudaMemset,
+ * torch.zeros).  Every call leaves the counters at zero again, a call that
+ * ends in WBMM_ERR_TIMEOUT included, and no call writes a counter word for
+ * anything else, so one workspace serves any number of later calls of any
+ * shape it is large enough for, graph replays included.  A call that ends in
+ * WBMM_ERR_CUDA may leave it dirty: zero it again.
+ * fp32 (and bf16 shapes outside the tensor-core kernels): the same counter
+ * region (left untouched), then fp32 partial tables, one per (channel, fixed
+ * chunk of windows), whose prior content does not matter.
  * The split depends only on the shape, the device's SM count and whether dX
  * is computed in the same call, so dT is bit-identical from run to run.
  * Calls that share a workspace must not overlap on the GPU.

@@ -67,12 +67,12 @@ def test_workspace_size_formula(lib):
     f = lib.wbmm_backward_workspace_bytes
     f.restype = ctypes.c_size_t
     f.argtypes = [ctypes.c_int] * 6
-    # bf16, tensor-core path: one partial table per (channel, CTA range)
-    # segment, at most n = C + min(256, tiles) - 1 of them, then one 32-bit
-    # arrival counter per channel (16-byte aligned).
+    # bf16, tensor-core path: a fixed region of 65536 arrival counters, then
+    # one partial table per (channel, CTA range) segment, at most
+    # n = C + min(256, tiles) - 1 of them.
     def tc(C, grid, tsz=729):
         n = C + grid - 1
-        return ((n * tsz + 3) // 4 * 4 + C) * 4
+        return (65536 + n * tsz) * 4
     # training workload: 64-window tiles of 32 two-window bands, 8 tiles per
     # channel, 2048 tiles -> 256 + 255 tables
     assert f(128, 256, 28, 28, 14, 1) == tc(256, 256)
@@ -83,7 +83,7 @@ def test_workspace_size_formula(lib):
     # 2 images of 112x112, w = 7: 64-window tiles of 4 bands, 8 tiles/channel
     assert f(2, 4, 112, 112, 7, 1) == tc(4, 32, 169)
     # fp32, CUDA-core path: chunks of 8 bands per channel
-    assert f(2, 3, 14, 28, 7, 0) == 3 * 1 * 169 * 4
+    assert f(2, 3, 14, 28, 7, 0) == (65536 + 3 * 1 * 169) * 4
     assert f(1, 1, 14, 15, 7, 1) == 0
 
 

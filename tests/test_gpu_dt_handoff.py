@@ -44,9 +44,9 @@ def workspace(B, C, H, W, w):
     return torch.zeros(n, dtype=torch.float32, device=DEV)
 
 
-def counters(ws, C):
-    """The workspace's last C words: one arrival counter per channel."""
-    return ws[-C:].view(torch.int32)
+def counters(ws):
+    """The workspace's counter region (one arrival counter per channel)."""
+    return ws[:wb.WBMM_DT_COUNTER_WORDS].view(torch.int32)
 
 
 def check_dt(dT, x, dy, w, what, channels=None):
@@ -64,13 +64,29 @@ def test_consecutive_calls_share_a_workspace(shape):
         x, dy = gen((B, C, H, W), 100 + 2 * call), gen((B, C, H, W), 101 + 2 * call)
         if call == 2:
             # partial tables left by the previous call must never be read
-            ws[:-C].fill_(float("nan"))
+            ws[wb.WBMM_DT_COUNTER_WORDS:].fill_(float("nan"))
         wb.wbmm_backward(x, None, dy, None, dT, ws, w)
         torch.cuda.synchronize()
         assert wb.wbmm_get_device_status() == 0
-        assert torch.all(counters(ws, C) == 0), "counters not reset"
+        assert torch.all(counters(ws) == 0), "counters not reset"
         assert torch.isfinite(dT).all()
         check_dt(dT, x, dy, w, "dT, call %d" % call)
+
+
+def test_one_workspace_serves_calls_of_different_shapes():
+    # the counter words are the same for every shape: calls of other shapes
+    # that wrote partial tables into the same buffer leave them zero
+    n = max(wb.wbmm_backward_workspace_bytes(*s, torch.bfloat16) for s in SPLIT_SHAPES) // 4
+    ws = torch.zeros(n, dtype=torch.float32, device=DEV)
+    for rnd in range(2):
+        for i, (B, C, H, W, w) in enumerate(SPLIT_SHAPES):
+            x, dy = gen((B, C, H, W), 140 + 4 * rnd + 2 * i), gen((B, C, H, W), 141 + 4 * rnd + 2 * i)
+            dT = torch.full((C, (2 * w - 1) ** 2), float("nan"), dtype=torch.float32, device=DEV)
+            wb.wbmm_backward(x, None, dy, None, dT, ws, w)
+            torch.cuda.synchronize()
+            assert wb.wbmm_get_device_status() == 0
+            assert torch.all(counters(ws) == 0), "counters not reset"
+            check_dt(dT, x, dy, w, "shape %d, round %d" % (i, rnd))
 
 
 @pytest.mark.parametrize("shape", SPLIT_SHAPES + [BOTH_SHAPE], ids=lambda s: "x".join(map(str, s)))
@@ -103,7 +119,7 @@ def test_graph_replay_with_new_inputs(shape):
         g.replay()
         torch.cuda.synchronize()
         assert wb.wbmm_get_device_status() == 0
-        assert torch.all(counters(ws, C) == 0), "counters not reset"
+        assert torch.all(counters(ws) == 0), "counters not reset"
         check_dt(dT, x, dy, w, "replay %d" % rep, channels)
         if both:
             xs, gs, Ts = to_np(x[:2, channels]), to_np(dy[:2, channels]), to_np(T[channels])

@@ -27,10 +27,13 @@ if not torch.cuda.is_available():
 import oracle  # noqa: E402
 import windowed_matmul_conv_b200 as wb  # noqa: E402
 
+# in this order, each shape's calls follow the previous shape's in the same
+# array: a CUDA-core call between tensor-core calls must leave the arrival
+# counters intact
 SHAPES = [
     (9, 3, 56, 56, 14, torch.bfloat16),   # tensor-core path, several tiles
-    (3, 2, 40, 40, 5, torch.bfloat16),    # odd window size
     (2, 3, 14, 28, 7, torch.float32),     # CUDA-core fp32 path
+    (3, 2, 40, 40, 5, torch.bfloat16),    # odd window size, another shape
 ]
 
 

@@ -33,6 +33,8 @@ if not os.path.exists(LIB_PATH):
 _lib = ctypes.CDLL(LIB_PATH)
 
 WBMM_F32, WBMM_BF16 = 0, 1
+# 32-bit arrival counters at the start of a table-gradient workspace
+WBMM_DT_COUNTER_WORDS = 65536
 STATUS_NAMES = {0: "WBMM_OK", 1: "WBMM_ERR_INVALID_ARG", 2: "WBMM_ERR_SHAPE",
                 3: "WBMM_ERR_DTYPE", 4: "WBMM_ERR_ALIGNMENT", 5: "WBMM_ERR_UNSUPPORTED",
                 6: "WBMM_ERR_WORKSPACE", 7: "WBMM_ERR_CUDA", 8: "WBMM_ERR_TIMEOUT"}

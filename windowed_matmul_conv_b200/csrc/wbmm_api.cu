@@ -119,12 +119,14 @@ size_t map_bytes(const Geom& g, wbmm_dtype dt)
     return (size_t)g.B * g.C * g.H * g.W * elem_size(dt);
 }
 
-// Workspace floats the backward will use for this shape and dtype.
+// Workspace floats the backward will use for this shape and dtype.  Every
+// workspace starts with the tensor-core path's counter region, so a buffer
+// shared by calls of both paths never has its counters overwritten.
 long long dt_workspace_floats(const Geom& g, wbmm_dtype dt)
 {
     if (dt == WBMM_BF16 && tc_dt_supported(g))
         return tc_dt_workspace_floats(g);
-    return (long long)g.C * simt_dt_chunks(g) * g.tsz;
+    return WBMM_DT_COUNTER_WORDS + (long long)g.C * simt_dt_chunks(g) * g.tsz;
 }
 
 }  // namespace
@@ -295,10 +297,11 @@ wbmm_status wbmm_backward(const void* x, const void* T, const void* dY, void* dX
             const bool after_dx = dX != nullptr;
             st = from_cuda(tc_dt_launch(g, x, dY, part, dT, after_dx, Lt));
         } else {
-            st = from_cuda(simt_dt_launch(g, dt == WBMM_BF16, x, dY, part, L));
+            float* chunks = part + WBMM_DT_COUNTER_WORDS;
+            st = from_cuda(simt_dt_launch(g, dt == WBMM_BF16, x, dY, chunks, L));
             if (st != WBMM_OK)
                 return st;
-            st = from_cuda(dt_finalize_launch(C, g.tsz, simt_dt_chunks(g), part, dT, L));
+            st = from_cuda(dt_finalize_launch(C, g.tsz, simt_dt_chunks(g), chunks, dT, L));
         }
     }
     return st;

@@ -78,10 +78,10 @@ cudaError_t tc_cached_launch(const Geom& g, const void* x, const void* M, void* 
                              const Launch& L);
 
 // tcgen05 table gradient: one contiguous tile range per CTA.  The workspace
-// (tc_dt_workspace_floats floats) holds the fp32 partial tables of channels
-// split between CTAs, then one 32-bit arrival counter per channel (its last C
-// words), which must be zero before the first launch; every launch leaves
-// them zero.
+// (tc_dt_workspace_floats floats) starts with WBMM_DT_COUNTER_WORDS 32-bit
+// arrival counters (one per channel; zero before the first launch, and every
+// launch leaves them zero), followed by the fp32 partial tables of channels
+// split between CTAs.
 // after_dx: the previous launch on the stream is the same backward call's
 // input-gradient kernel (which reads dY and T and writes only dX), so the
 // kernel need not wait for it to finish.  The grid is min(L.num_sms, 256,

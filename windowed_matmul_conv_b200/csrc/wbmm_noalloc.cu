@@ -8,11 +8,15 @@
 // the same dT as wbmm_backward, with its per-chunk partial tables in a
 // file-scope device array instead of a workspace argument.
 //
-// The array is kStaticPartials floats (4 MiB).  Every GPU that loads this
-// library holds it until the process exits.  All calls share it; each call
-// overwrites every entry it reads, so nothing has to start at zero, but calls
-// whose work overlaps on the GPU (different streams, or devices sharing
-// nothing but the host thread) race on it and must be ordered by the caller.
+// The array is kStaticPartials floats (4 MiB), laid out like a workspace of
+// wbmm_backward: its first words are the tensor-core path's per-channel
+// arrival counters, which start at zero (a __device__ array is zero-filled
+// when the library loads) and which every call leaves at zero; the partial
+// tables after them are overwritten before they are read.  Every GPU that
+// loads this library holds it until the process exits.  All calls share it,
+// so calls whose work overlaps on the GPU (different streams, or devices
+// sharing nothing but the host thread) race on it and must be ordered by the
+// caller.
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -84,7 +88,8 @@ extern "C" WBMM_API wbmm_status wbmm_backward_dt_static(const void* x, const voi
     }
     // Same partial-table split as wbmm_backward, checked against the array.
     const bool tc = dt == WBMM_BF16 && tc_dt_supported(g);
-    const long long need = tc ? tc_dt_workspace_floats(g) : (long long)C * simt_dt_chunks(g) * g.tsz;
+    const long long need = tc ? tc_dt_workspace_floats(g)
+                              : WBMM_DT_COUNTER_WORDS + (long long)C * simt_dt_chunks(g) * g.tsz;
     if ((unsigned long long)need > kStaticPartials)
         return WBMM_ERR_WORKSPACE;
 
@@ -100,9 +105,11 @@ extern "C" WBMM_API wbmm_status wbmm_backward_dt_static(const void* x, const voi
     if (tc) {
         e = tc_dt_launch(g, x, dY, part, dT, false, L);
     } else {
-        e = simt_dt_launch(g, dt == WBMM_BF16, x, dY, part, L);
+        // the CUDA-core path's partial tables also sit after the counters
+        float* chunks = part + WBMM_DT_COUNTER_WORDS;
+        e = simt_dt_launch(g, dt == WBMM_BF16, x, dY, chunks, L);
         if (e == cudaSuccess)
-            e = dt_finalize_launch(C, g.tsz, simt_dt_chunks(g), part, dT, L);
+            e = dt_finalize_launch(C, g.tsz, simt_dt_chunks(g), chunks, dT, L);
     }
     if (e == cudaErrorInvalidConfiguration)
         return WBMM_ERR_UNSUPPORTED;

@@ -13,15 +13,16 @@
 // into its own fp32 partial table.  A channel inside one CTA's range is
 // written to dT directly.  A channel split between CTAs k0 < ... < k1 is
 // finished by whichever of them arrives last: each writes its segment's
-// partial table (at index c + k of the workspace: ranges are ordered, so the
-// index is unique) and then adds one to the channel's arrival counter
+// partial table (at index c + k of the workspace's tables: ranges are
+// ordered, so the index is unique) and then adds one to the channel's arrival
+// counter
 // (acquire-release, device scope); the CTA that sees the count reach
 // k1 - k0 + 1 adds the partial tables in CTA order k0, ..., k1 into dT and
 // sets the counter back to zero.  No CTA ever waits for another, so the grid
 // need not be co-resident, and a counter can only reach its final count
 // within one launch: a re-launch with the same arguments (a replayed graph)
 // never sees the previous launch's partials as ready.  Every counter starts
-// at zero (the workspace's counter words must be zero before the first call)
+// at zero (the workspace's counter region must be zero before its first use)
 // and every launch leaves it zero, the aborted ones included, since each CTA
 // arrives once per split channel whether or not its waits succeeded.  Every
 // sum runs in a fixed order, so the result is bit-identical from run to run
@@ -43,6 +44,7 @@
 #include <cuda_bf16.h>
 
 #include "ptx_sm100.cuh"
+#include "wbmm.h"
 #include "tc_common.cuh"
 #include "wbmm_internal.h"
 
@@ -584,13 +586,6 @@ constexpr int kDtMaxGrid = 256;
 
 long long tc_dt_partials_impl(const Geom& g);
 
-// Float offset of the arrival counters in the workspace (after the partial
-// tables, rounded up to 16 bytes).
-long long dt_counters_offset(const Geom& g)
-{
-    return (tc_dt_partials_impl(g) * g.tsz + 3) / 4 * 4;
-}
-
 int dt_tiles_per_channel(const Geom& g)
 {
     const int bpt = dt_nt_for(g.w) / g.nw;
@@ -625,8 +620,8 @@ cudaError_t dt_launch_ws(const Geom& g, const void* x, const void* dy, float* wo
     TcDtParams P;
     P.x = static_cast<const uint16_t*>(x);
     P.dy = static_cast<const uint16_t*>(dy);
-    P.partials = workspace;
-    P.counters = reinterpret_cast<unsigned int*>(workspace + dt_counters_offset(g));
+    P.counters = reinterpret_cast<unsigned int*>(workspace);
+    P.partials = workspace + WBMM_DT_COUNTER_WORDS;
     P.dT = dT;
     P.C = g.C; P.H = g.H; P.W = g.W; P.nh = g.nh; P.nw = g.nw;
     P.bpt = F::NT / g.nw;
@@ -687,6 +682,8 @@ bool tc_dt_supported(const Geom& g)
         return false;
     if (g.bands * (long long)g.C >= (1ll << 31))
         return false;
+    if (g.C > WBMM_DT_COUNTER_WORDS)
+        return false;
     return true;
 }
 
@@ -702,9 +699,10 @@ long long tc_dt_tiles(const Geom& g)
 
 long long tc_dt_workspace_floats(const Geom& g)
 {
-    // partial tables, then one 32-bit arrival counter per channel (16-byte
-    // aligned), the workspace's last C words
-    return dt_counters_offset(g) + g.C;
+    // a fixed region of arrival counters (one per channel, the same words for
+    // every shape, so a workspace shared by calls of different shapes keeps
+    // them zero), then the partial tables
+    return WBMM_DT_COUNTER_WORDS + tc_dt_partials(g) * g.tsz;
 }
 
 cudaError_t tc_dt_launch(const Geom& g, const void* x, const void* dy, float* partials, float* dT,
