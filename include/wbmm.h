@@ -241,6 +241,31 @@ WBMM_API wbmm_status wbmm_wait_selftest(unsigned long long cycles, void *stream)
 WBMM_API unsigned long long wbmm_launch_count(void);
 
 /*
+ * Test-only settings, off by default, for exercising failure handling
+ * without faulting the GPU (the library's own tests use them; a normal
+ * caller never needs them).  No counterpart in the paper.
+ *   WBMM_DEBUG_SKIP_LOAD_WINDOW_MAJOR, value t >= 0: in the next launch of
+ *     the window-major tensor-core kernel (wbmm_forward, or the input
+ *     gradient of wbmm_backward, w <= 16), the load producer of CTA 0 skips
+ *     its t-th tile; the consumer's bounded wait for it runs out, the kernel
+ *     abandons its work, drains its copies and MMAs, releases its tensor
+ *     memory and returns, and wbmm_get_device_status() reports
+ *     WBMM_ERR_TIMEOUT.  The outputs of that call are undefined.  Consumed by
+ *     that launch; value < 0 clears it.
+ *   WBMM_DEBUG_SKIP_LOAD_TABLE_GRAD: the same for the next launch of the
+ *     tensor-core table-gradient kernel.
+ *   WBMM_DEBUG_RING_CAP, value n: the window-major and table-gradient
+ *     kernels use at most n load slots (0 restores the default, as many as
+ *     fit); results do not depend on it.
+ * Pair a skip with a short wait budget (wbmm_set_wait_budget).  Process-wide;
+ * not for concurrent use.  Returns WBMM_ERR_INVALID_ARG for an unknown `what`.
+ */
+#define WBMM_DEBUG_SKIP_LOAD_WINDOW_MAJOR 1
+#define WBMM_DEBUG_SKIP_LOAD_TABLE_GRAD 2
+#define WBMM_DEBUG_RING_CAP 3
+WBMM_API wbmm_status wbmm_debug_set(int what, int value);
+
+/*
  * Kernel family used by the most recent successful wbmm_forward,
  * wbmm_backward (input-gradient part) or wbmm_forward_cached call on this
  * host thread: 1 = tcgen05 tensor-core kernel, 2 = CUDA-core (SIMT) kernel.

@@ -42,7 +42,7 @@ EXPORTS = ("wbmm_forward", "wbmm_backward_workspace_bytes", "wbmm_backward",
            "wbmm_cache_matrices", "wbmm_reparam_merge", "wbmm_forward_cached", "wbmm_dw3x3",
            "wbmm_get_device_status", "wbmm_status_string", "wbmm_set_wait_budget",
            "wbmm_wait_selftest", "wbmm_launch_count", "wbmm_last_path",
-           "wbmm_backward_dt_static")
+           "wbmm_backward_dt_static", "wbmm_debug_set")
 
 _vp, _i, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
 _lib.wbmm_forward.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]
@@ -63,8 +63,10 @@ _lib.wbmm_wait_selftest.argtypes = [ctypes.c_ulonglong, _vp]
 _lib.wbmm_launch_count.argtypes = []
 _lib.wbmm_launch_count.restype = ctypes.c_ulonglong
 _lib.wbmm_last_path.argtypes = []
+_lib.wbmm_debug_set.argtypes = [_i, _i]
 for _f in ("wbmm_forward", "wbmm_backward", "wbmm_backward_dt_static", "wbmm_cache_matrices",
-           "wbmm_reparam_merge", "wbmm_forward_cached", "wbmm_dw3x3", "wbmm_get_device_status", "wbmm_wait_selftest", "wbmm_last_path"):
+           "wbmm_reparam_merge", "wbmm_forward_cached", "wbmm_dw3x3", "wbmm_get_device_status", "wbmm_wait_selftest", "wbmm_last_path",
+           "wbmm_debug_set"):
     getattr(_lib, _f).restype = _i
 
 
@@ -224,6 +226,14 @@ def wbmm_launch_count():
 
 def wbmm_last_path():
     return int(_lib.wbmm_last_path())
+
+
+# test-only settings of wbmm_debug_set (include/wbmm.h)
+WBMM_DEBUG_SKIP_LOAD_WINDOW_MAJOR, WBMM_DEBUG_SKIP_LOAD_TABLE_GRAD, WBMM_DEBUG_RING_CAP = 1, 2, 3
+
+
+def wbmm_debug_set(what, value):
+    _check(_lib.wbmm_debug_set(int(what), int(value)))
 
 
 # ------------------------------------------------------------ conveniences

@@ -31,6 +31,12 @@ std::mutex g_mu;
 DevInfo g_dev[kMaxDevices];
 std::atomic<unsigned long long> g_launches{0};
 std::atomic<unsigned long long> g_budget{kDefaultBudget};
+// Test-only settings (wbmm_debug_set): a tile whose load the producer of
+// CTA 0 skips in the next launch of a kernel family (-1: none), and a cap on
+// the load ring's depth (0: none).
+std::atomic<int> g_dbg_skip_toep{-1};
+std::atomic<int> g_dbg_skip_dt{-1};
+std::atomic<int> g_dbg_ring_cap{0};
 thread_local int t_last_path = 0;
 
 wbmm_status dev_info(DevInfo** out)
@@ -133,6 +139,13 @@ long long dt_workspace_floats(const Geom& g, wbmm_dtype dt)
 
 void note_launches(int n) { g_launches.fetch_add((unsigned long long)n); }
 
+int debug_take_skip(int family)
+{
+    return (family == 0 ? g_dbg_skip_toep : g_dbg_skip_dt).exchange(-1);
+}
+
+int debug_ring_cap() { return g_dbg_ring_cap.load(); }
+
 int launch_for_stream(void* stream, Launch* L) { return (int)make_launch(stream, L); }
 
 }  // namespace wbmm
@@ -163,6 +176,16 @@ void wbmm_set_wait_budget(unsigned long long cycles)
 }
 
 unsigned long long wbmm_launch_count(void) { return g_launches.load(); }
+
+wbmm_status wbmm_debug_set(int what, int value)
+{
+    switch (what) {
+    case WBMM_DEBUG_SKIP_LOAD_WINDOW_MAJOR: g_dbg_skip_toep.store(value < 0 ? -1 : value); return WBMM_OK;
+    case WBMM_DEBUG_SKIP_LOAD_TABLE_GRAD: g_dbg_skip_dt.store(value < 0 ? -1 : value); return WBMM_OK;
+    case WBMM_DEBUG_RING_CAP: g_dbg_ring_cap.store(value < 0 ? 0 : value); return WBMM_OK;
+    }
+    return WBMM_ERR_INVALID_ARG;
+}
 
 int wbmm_last_path(void) { return t_last_path; }
 

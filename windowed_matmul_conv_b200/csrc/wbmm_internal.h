@@ -135,4 +135,11 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 // current device; returns a wbmm_status code (0 on success).
 int launch_for_stream(void* stream, Launch* L);
 
+// Test-only settings of wbmm_debug_set.  debug_take_skip(family) returns the
+// tile (in CTA 0's order) whose load the next launch of the family skips and
+// clears it (-1: none; family 0 = window-major forward / input gradient,
+// 1 = table gradient); debug_ring_cap() caps the load ring (0: no cap).
+int debug_take_skip(int family);
+int debug_ring_cap();
+
 }  // namespace wbmm

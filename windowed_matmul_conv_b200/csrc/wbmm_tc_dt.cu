@@ -120,6 +120,7 @@ struct TcDtParams {
     int kimg;               // planes per tile when use_tmap
     int R;                  // raw ring depth (tiles)
     uint32_t off_raw, off_stage, off_stg, off_woff, off_bar;
+    int skip_seq;           // test only: CTA 0 skips this tile's load (-1: none)
     unsigned long long budget;
     int* status;
 };
@@ -251,6 +252,12 @@ __global__ void __launch_bounds__(kDtThreads, 1) wbmm_tc_dt_kernel(const __grid_
                 break;
             const DtTile t = it.get(P);
             uint8_t* slot = raw_base + (size_t)s * F::RAW_BYTES;
+            if (seq == P.skip_seq && blockIdx.x == 0) {
+                // test only: the slot is never armed, so the transform's
+                // bounded wait for it runs out
+                issued = seq + 1;
+                continue;
+            }
             if (P.use_tmap) {
                 if (lane == 0) {
                     mbar_arrive_expect_tx(&S.raw_full[s], 2u * P.kimg * WS * P.W * P.nh * 2);
@@ -571,6 +578,9 @@ DtLayout dt_layout()
     const uint32_t avail = kSmemMax - 1024 > L.off_raw ? kSmemMax - 1024 - L.off_raw : 0;
     int R = (int)(avail / F::RAW_BYTES);
     L.R = R < kDtRingMax ? R : kDtRingMax;
+    const int cap = debug_ring_cap();
+    if (cap >= 2 && L.R > cap)
+        L.R = cap;
     off = L.off_raw + (uint32_t)L.R * F::RAW_BYTES;
     L.total = align_up(off, 1024);
     // at least half the SM's shared memory: one CTA (and one 512-column TMEM
@@ -612,7 +622,7 @@ cudaError_t dt_launch_ws(const Geom& g, const void* x, const void* dy, float* wo
     if (!(configured & (1ull << (dev & 63)))) {
         cudaError_t e = cudaFuncSetAttribute(wbmm_tc_dt_kernel<WS>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)lay.total);
+                                             (int)kSmemMax);
         if (e != cudaSuccess)
             return e;
         configured |= 1ull << (dev & 63);
@@ -662,6 +672,7 @@ cudaError_t dt_launch_ws(const Geom& g, const void* x, const void* dy, float* wo
     P.off_woff = lay.off_woff; P.off_bar = lay.off_bar;
     P.budget = L.budget;
     P.status = L.status;
+    P.skip_seq = debug_take_skip(1);
     cudaError_t e = launch_pdl(wbmm_tc_dt_kernel<WS>, dim3(grid), dim3(kDtThreads), lay.total,
                                L.stream, P);
     if (e != cudaSuccess)

@@ -116,6 +116,7 @@ struct TcToepParams {
     int use_tmap;
     int kimg_sub;           // planes per half tile when use_tmap
     uint32_t off_out, off_q, off_raw, off_woff, off_bar, off_tst;
+    int skip_seq;           // test only: CTA 0 skips this tile's load (-1: none)
     unsigned long long budget;
     int* status;
 };
@@ -304,10 +305,10 @@ __global__ void __launch_bounds__(kToepThreads, 1)
 
     if (warp == 0) {
         // ------------------------------------------------------ producer
-        // The first two tables' loads are issued before any tile's, so that
-        // they are not queued behind every CTA's ring fill (the first MMA
-        // needs Q).
-        named_bar_sync(5, 32 + kToepEpiWarps * 32);
+        // The first tile's loads go out at once, beside the epilogue warps'
+        // loads of the first two tables; the rest of the ring waits until
+        // those tables have arrived, so that they are not queued behind every
+        // CTA's ring fill (the first MMA needs Q).
         int issued = 0;
         bool go = true;
         for (int seq = 0; seq < n_it && go; ++seq) {
@@ -324,7 +325,10 @@ __global__ void __launch_bounds__(kToepThreads, 1)
                 }
                 const BandTile st = toep_half(P, t, h);
                 uint8_t* slot = raw_base + (size_t)s * P.sub_bytes;
-                if (st.nb == 0) {
+                if (seq == P.skip_seq && blockIdx.x == 0) {
+                    // test only: the slot is never armed, so the transform's
+                    // bounded wait for it runs out
+                } else if (st.nb == 0) {
                     if (lane == 0)
                         mbar_arrive_expect_tx(&S.raw_full[s], 0);
                 } else if (P.use_tmap) {
@@ -349,7 +353,11 @@ __global__ void __launch_bounds__(kToepThreads, 1)
                 }
                 issued = ss + 1;
             }
+            if (seq == 0)
+                named_bar_sync(5, 32 + kToepEpiWarps * 32);
         }
+        if (n_it == 0)
+            named_bar_sync(5, 32 + kToepEpiWarps * 32);
         // Drain: every issued copy lands before the CTA can exit.
         if (lane == 0) {
             for (int s = 0; s < R && s < issued; ++s) {
@@ -692,6 +700,9 @@ bool toep_layout_n(const Geom& g, int nout, ToepLayout& L)
     int R = (int)(avail / L.sub_bytes);
     if (R > kToepRing)
         R = kToepRing;
+    const int cap = debug_ring_cap();
+    if (cap >= 2 && R > cap)
+        R = cap;
     L.R = R;
     if (R < 2)
         return false;
@@ -755,6 +766,7 @@ cudaError_t toep_launch_ws(const Geom& g, const void* x, const void* T, void* y,
     P.off_woff = lay.off_woff; P.off_bar = lay.off_bar; P.off_tst = lay.off_tst;
     P.budget = L.budget;
     P.status = L.status;
+    P.skip_seq = debug_take_skip(0);
     int grid = L.num_sms;
     if (grid > P.items)
         grid = P.items;
