@@ -5,9 +5,9 @@ synthetic input.  Default workload (the training step): B128 C256 28x28, w=14,
 bf16 -- forward y = WBMM(x; T), then the backward dX = M^T dY and the table
 gradient dT, all through the C ABI.  Other workloads (--workload): fwd
 (B64 C128 56x56 w14), sweep7 / sweep14 / sweep28 (B32 C256 112x112), cached
-(B8 C96 224x224 w14, cached matrices + 3x3 mixing), fwd32 (the fp32 forward
-of the fwd shape) and reparam (the cached shape through one matrix merged from a
-14x14 and a 7x7 table).
+(B8 C96 224x224 w14, cached matrices + 3x3 mixing), fwd32 / train32 / cached32
+(the fp32 path on the fwd, train and cached shapes) and reparam (the cached
+shape through one matrix merged from a 14x14 and a 7x7 table).
 
 Multi-GPU (torchrun): every rank owns its own block of channels with the
 per-GPU workload above (weak scaling); channels are independent, so the hot
@@ -40,6 +40,8 @@ WORKLOADS = {
     "train": "train_bf16",
     "fwd": "fwd_bf16",
     "fwd32": "fwd_f32",
+    "train32": "train_f32",
+    "cached32": "hires_cached_dw_f32",
     "sweep7": "sweep_w7",
     "sweep14": "sweep_w14",
     "sweep28": "sweep_w28",
@@ -208,7 +210,8 @@ class Arm:
         self.T = d["T"].to(dev)
         if wl.kind == "train":
             self.dT = torch.empty((wl.C, wl.t), dtype=torch.float32, device=dev)
-            nbytes = wb.wbmm_backward_workspace_bytes(wl.B, wl.C, wl.H, wl.W, wl.w, torch.bfloat16)
+            nbytes = wb.wbmm_backward_workspace_bytes(wl.B, wl.C, wl.H, wl.W, wl.w,
+                                                      synth.torch_dtype(wl.dtype))
             # zero-filled once: the table gradient's arrival counters start at zero
             self.ws = torch.zeros(max(1, nbytes // 4), dtype=torch.float32, device=dev)
         if wl.kind == "reparam":
@@ -244,7 +247,9 @@ class Arm:
         if self.wl.kind == "train":
             # one gradient per call: each kernel alone on the whole device
             return ["backward_dx", "backward_dt"]
-        return ["forward_cached_dw3x3"] if self.wl.kind == "cached_dw" else []
+        # the fused launch covers bf16 maps only
+        return (["forward_cached_dw3x3"] if self.wl.kind == "cached_dw" and self.wl.dtype == "bf16"
+                else [])
 
     def calls(self):
         """The step as a user issues it: the training step is one forward

@@ -64,6 +64,10 @@ WORKLOADS = {
     "sweep_w28": Workload("sweep_w28", 32, 256, 112, 112, 28, "bf16", "normal", "forward"),
     "hires_cached_dw": Workload("hires_cached_dw", 8, 96, 224, 224, 14, "bf16", "normal",
                                 "cached_dw"),
+    # the fp32 path (CUDA cores) on the training and high-res cached shapes
+    "train_f32": Workload("train_f32", 128, 256, 28, 28, 14, "f32", "truncated", "train"),
+    "hires_cached_dw_f32": Workload("hires_cached_dw_f32", 8, 96, 224, 224, 14, "f32", "normal",
+                                    "cached_dw"),
     # inference with a 14x14 and a 7x7 branch folded into one matrix
     "hires_reparam": Workload("hires_reparam", 8, 96, 224, 224, 14, "bf16", "normal", "reparam"),
 }
