@@ -488,3 +488,88 @@ def test_full_size_cached_dw_sampled():
     # the forward row bound
     zb = oracle.dw3x3(forward_rowbound(xs, Ts, wl.w), np.abs(Ks))
     check_bf16(to_np(z[bs][:, cs]), zref, zb, "hires z")
+
+
+def test_full_size_fp32_training_step_sampled():
+    # the fp32 path (CUDA cores) on the training workload, as bench.py
+    # --workload train32 runs it: sampled planes for y and dX, whole sampled
+    # channels for dT
+    wl = synth.WORKLOADS["train_f32"]
+    d = synth.draw(wl, seed=0)
+    x, T, dy = d["x"].to(DEV), d["T"].to(DEV), d["dY"].to(DEV)
+    y = run_forward(x, T, wl.w)
+    dX, dT = wb.backward(x, T, dy, wl.w)
+    torch.cuda.synchronize()
+    assert wb.wbmm_get_device_status() == 0
+    assert wb.wbmm_last_path() == 2
+    bs, cs = sample_planes(wl.B, wl.C)
+    xs, gs, Ts = to_np(d["x"][bs][:, cs]), to_np(d["dY"][bs][:, cs]), to_np(d["T"][cs])
+    check_f32(to_np(y[bs][:, cs]), oracle.forward(xs, Ts, wl.w),
+              oracle.forward(np.abs(xs), np.abs(Ts), wl.w), "train32 y")
+    check_f32(to_np(dX[bs][:, cs]), oracle.backward_dx(gs, Ts, wl.w),
+              oracle.backward_dx(np.abs(gs), np.abs(Ts), wl.w), "train32 dX")
+    xc, gc = to_np(d["x"][:, cs]), to_np(d["dY"][:, cs])
+    check_f32(to_np(dT[cs]), oracle.backward_dt(xc, gc, wl.w),
+              oracle.backward_dt(np.abs(xc), np.abs(gc), wl.w), "train32 dT")
+
+
+def test_full_size_fp32_cached_dw_sampled():
+    wl = synth.WORKLOADS["hires_cached_dw_f32"]
+    d = synth.draw(wl, seed=0)
+    x, T, K = d["x"].to(DEV), d["T"].to(DEV), d["K"].to(DEV)
+    M = wb.cache_matrices(T, wl.w)
+    y = wb.forward_cached(x, M, wl.w)
+    z = wb.dw3x3(y, K)
+    torch.cuda.synchronize()
+    assert wb.wbmm_get_device_status() == 0
+    bs, cs = sample_planes(wl.B, wl.C)
+    xs, Ts, Ks = to_np(d["x"][bs][:, cs]), to_np(d["T"][cs]), to_np(d["K"][cs])
+    yref = oracle.forward(xs, Ts, wl.w)
+    yabs = oracle.forward(np.abs(xs), np.abs(Ts), wl.w)
+    check_f32(to_np(y[bs][:, cs]), yref, yabs, "cached32 y")
+    # the 3x3 of the GPU's own y: z's error against that is the stencil's
+    # fp32 accumulation alone
+    yg = to_np(y[bs][:, cs])
+    check_f32(to_np(z[bs][:, cs]), oracle.dw3x3(yg, Ks), oracle.dw3x3(np.abs(yg), np.abs(Ks)),
+              "cached32 z")
+
+
+def test_full_size_reparam_sampled():
+    # the high-resolution shape through one matrix merged from a 14x14 and a
+    # 7x7 table, as bench.py --workload reparam runs it
+    wl = synth.WORKLOADS["hires_reparam"]
+    k = synth.REPARAM_SMALL_WINDOW
+    d = synth.draw(wl, seed=0)
+    x, T, Tk = d["x"].to(DEV), d["T"].to(DEV), d["Tk"].to(DEV)
+    M = wb.reparam_merge(T, Tk, wl.w, k)
+    y = wb.forward_cached(x, M, wl.w)
+    torch.cuda.synchronize()
+    assert wb.wbmm_get_device_status() == 0
+    bs, cs = sample_planes(wl.B, wl.C)
+    xs = to_np(d["x"][bs][:, cs])
+    ref = oracle.forward(xs, to_np(d["T"][cs]), wl.w) + oracle.forward(xs, to_np(d["Tk"][cs]), k)
+    Mn = to_np(M[cs])
+    rn = np.sqrt((Mn ** 2).sum(axis=2)).reshape(len(cs), wl.w, wl.w)
+    bound = window_norms(xs, wl.w) * np.tile(rn, (1, wl.H // wl.w, wl.W // wl.w))[None]
+    check_bf16(to_np(y[bs][:, cs]), ref, bound, "reparam y")
+
+
+@pytest.mark.parametrize("shape", [(3, 2, 56, 56, 14), (2, 3, 35, 70, 7), (1, 2, 15, 45, 5),
+                                   (5, 1, 42, 28, 14)], ids=lambda s: "x".join(map(str, s)))
+def test_fp32_cached_forward_equals_table_forward(shape):
+    # both CUDA-core kernels sum each output's d products in (r, s) order
+    # with fused multiply-adds, and the cached matrix holds exact copies of
+    # table entries: the results agree bit for bit; also checked against the
+    # oracle (window counts that are not multiples of the 64-window tile)
+    B, C, H, W, w = shape
+    x = gen((B, C, H, W), 40, torch.float32)
+    T = gen((C, (2 * w - 1) ** 2), 41, torch.float32, 0.02)
+    M = wb.cache_matrices(T, w)
+    yc = wb.forward_cached(x, M, w)
+    yt = wb.forward(x, T, w)
+    torch.cuda.synchronize()
+    assert wb.wbmm_get_device_status() == 0
+    assert torch.equal(yc, yt)
+    xr, Tr = to_np(x), to_np(T)
+    check_f32(to_np(yc), oracle.forward(xr, Tr, w), oracle.forward(np.abs(xr), np.abs(Tr), w),
+              "fp32 cached")

@@ -4,6 +4,8 @@
 // mixing and the bounded-wait self-test.
 #include <cuda_bf16.h>
 
+#include <type_traits>
+
 #include <utility>
 
 #include "dw_common.cuh"
@@ -71,6 +73,139 @@ __global__ void simt_fwd_kernel(const TIn* __restrict__ x, const TIn* __restrict
             }
         }
         yb[p * W + j * w + q] = from_f<TIn>(acc);
+    }
+}
+
+// ------------------------------------------------ forward, cached matrices
+// Register-tiled form of the cached-matrix sums (d = w*w <= 196): a block
+// holds M_c^T (rows v, d padded to DP = roundup(d, 8) columns u) and a tile
+// of whole bands (at most 64 windows) X[v][n] in shared memory as fp32, the
+// tile stored with a row stride of 68 floats so that the transposing writes
+// of the band loads meet few bank conflicts; thread (ug, ng) keeps the 8 x 4
+// outputs (u = 8ug.., n = 4ng..) in registers and, for each v, loads two
+// float4 of M and one of X for 32 fused multiply-adds.  Loads and stores
+// walk band rows, one lane per element.  Each output is one fp32 sum in
+// v = (r, s) order, as in simt_fwd_kernel, so the results are bit-identical
+// to it.  Blocks take contiguous runs of one channel's tiles, so M_c is
+// loaded once per run.
+constexpr int kCachedNT = 64;       // windows per tile, at most
+constexpr int kCachedXS = 68;       // row stride of the tile in shared memory
+constexpr size_t kCachedSmemMax = 232448;       // the per-block maximum on sm_100
+
+template <typename TIn>
+__global__ void __launch_bounds__(400, 1)
+    simt_cached_kernel(const TIn* __restrict__ x, const TIn* __restrict__ M, TIn* __restrict__ y,
+                       int C, int H, int W, int w, int nh, int nw, long long bands, int bpt,
+                       int ntiles, int tpb, int G)
+{
+    extern __shared__ __align__(16) float smc[];
+    const int d = w * w, DP = (d + 7) / 8 * 8;
+    float* MT = smc;                              // [d][DP]
+    float* XS = smc + (size_t)d * DP;             // [d][kCachedXS], then Y[u][n]
+    grid_dep_wait();
+    grid_dep_launch();
+    const int c = blockIdx.x / G, gidx = blockIdx.x - (blockIdx.x / G) * G;
+    const int t0 = gidx * tpb, t1 = t0 + tpb < ntiles ? t0 + tpb : ntiles;
+    if (t0 >= t1)
+        return;
+    const int tid = threadIdx.x, nthr = blockDim.x;
+    const int lane = tid & 31, warp = tid >> 5, nwarps = nthr >> 5;
+    const TIn* Mc = M + (long long)c * d * d;
+    // fp32 operands go to shared memory as asynchronous 4-byte copies, all of
+    // a tile's in flight at once; bf16 ones are widened through registers
+    constexpr bool kAsync = std::is_same<TIn, float>::value;
+    for (int e = tid; e < d * d; e += nthr) {
+        const int u = e / d, v = e - (e / d) * d;
+        if constexpr (kAsync)
+            cp_async_4(smem_u32(MT + v * DP + u), Mc + e);
+        else
+            MT[v * DP + u] = to_f(Mc[e]);
+    }
+    const int ug = tid >> 4, ng = tid & 15;
+    const bool active = 8 * ug < d;
+    for (int t = t0; t < t1; ++t) {
+        const long long g0 = (long long)t * bpt;
+        const int nb = bands - g0 < bpt ? (int)(bands - g0) : bpt;
+        __syncthreads();        // M_c written; the previous tile's outputs stored
+        // zero the windows past the tile's last band (read by the register
+        // tiles, never stored)
+        for (int e = tid; e < d * kCachedNT; e += nthr) {
+            const int v = e >> 6, n = e & (kCachedNT - 1);
+            if (n >= nb * nw)
+                XS[v * kCachedXS + n] = 0.0f;
+        }
+        for (int row = warp; row < nb * w; row += nwarps) {
+            const int kb = row / w, r = row - (row / w) * w;
+            const long long gb = g0 + kb;
+            const long long b = gb / nh;
+            const int i = (int)(gb - b * nh);
+            const TIn* src = x + ((b * C + c) * H + (long long)i * w + r) * W;
+            for (int col = lane; col < W; col += 32) {
+                const int j = col / w, sidx = col - (col / w) * w;
+                float* dst = XS + (r * w + sidx) * kCachedXS + kb * nw + j;
+                if constexpr (kAsync)
+                    cp_async_4(smem_u32(dst), src + col);
+                else
+                    *dst = to_f(src[col]);
+            }
+        }
+        if constexpr (kAsync)
+            cp_async_wait_all();
+        __syncthreads();
+        float acc[8][4];
+#pragma unroll
+        for (int a = 0; a < 8; ++a)
+#pragma unroll
+            for (int bq = 0; bq < 4; ++bq)
+                acc[a][bq] = 0.0f;
+        if (active) {
+            // the operands of v + 1 are loaded while the 32 multiply-adds of
+            // v run, so the shared-memory latency is not exposed
+            const float* mp = MT + 8 * ug;
+            const float* xp = XS + 4 * ng;
+            float4 m0 = *reinterpret_cast<const float4*>(mp);
+            float4 m1 = *reinterpret_cast<const float4*>(mp + 4);
+            float4 xv = *reinterpret_cast<const float4*>(xp);
+#pragma unroll 2
+            for (int v = 0; v < d; ++v) {
+                const int vn = v + 1 < d ? v + 1 : v;
+                const float4 n0 = *reinterpret_cast<const float4*>(mp + vn * DP);
+                const float4 n1 = *reinterpret_cast<const float4*>(mp + vn * DP + 4);
+                const float4 nx = *reinterpret_cast<const float4*>(xp + vn * kCachedXS);
+                const float mv[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+                const float xs[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+                for (int a = 0; a < 8; ++a)
+#pragma unroll
+                    for (int bq = 0; bq < 4; ++bq)
+                        acc[a][bq] = __fmaf_rn(mv[a], xs[bq], acc[a][bq]);
+                m0 = n0;
+                m1 = n1;
+                xv = nx;
+            }
+        }
+        __syncthreads();        // every thread is done reading XS
+        if (active) {
+#pragma unroll
+            for (int a = 0; a < 8; ++a) {
+                const int u = 8 * ug + a;
+                if (u < d)
+                    *reinterpret_cast<float4*>(XS + u * kCachedXS + 4 * ng) =
+                        make_float4(acc[a][0], acc[a][1], acc[a][2], acc[a][3]);
+            }
+        }
+        __syncthreads();
+        for (int row = warp; row < nb * w; row += nwarps) {
+            const int kb = row / w, p = row - (row / w) * w;
+            const long long gb = g0 + kb;
+            const long long b = gb / nh;
+            const int i = (int)(gb - b * nh);
+            TIn* dst = y + ((b * C + c) * H + (long long)i * w + p) * W;
+            for (int col = lane; col < W; col += 32) {
+                const int j = col / w, q = col - (col / w) * w;
+                dst[col] = from_f<TIn>(XS[(p * w + q) * kCachedXS + kb * nw + j]);
+            }
+        }
     }
 }
 
@@ -540,6 +675,41 @@ cudaError_t simt_fwd_launch(const Geom& g, AMode mode, bool is_bf16, const void*
                                       is_bf16, x, src, y, L);
         if (e != cudaErrorInvalidValue)
             return e;
+    }
+    if (mode == kCached && g.w >= 3 && g.w <= 14 && g.nw <= kCachedNT) {
+        const int d = g.d, DP = (d + 7) / 8 * 8;
+        const size_t csmem = ((size_t)d * DP + (size_t)d * kCachedXS) * 4;
+        const int bpt = kCachedNT / g.nw;         // whole bands per tile
+        const int ntiles = (int)((g.bands + bpt - 1) / bpt);
+        if (csmem <= kCachedSmemMax && ntiles > 0) {
+            // about two blocks' worth of runs per SM, M_c loaded once per run
+            int G = (2 * L.num_sms + g.C - 1) / g.C;
+            if (G > ntiles)
+                G = ntiles;
+            const int tpb = (ntiles + G - 1) / G;
+            const dim3 grid((unsigned)(g.C * G)), block((unsigned)(DP / 8 * 16));
+            cudaError_t e;
+            if (is_bf16) {
+                using E = __nv_bfloat16;
+                e = set_smem(simt_cached_kernel<E>, csmem);
+                if (e == cudaSuccess)
+                    e = launch_pdl(simt_cached_kernel<E>, grid, block, csmem, L.stream,
+                                   static_cast<const E*>(x), static_cast<const E*>(src),
+                                   static_cast<E*>(y), g.C, g.H, g.W, g.w, g.nh, g.nw, g.bands,
+                                   bpt, ntiles, tpb, G);
+            } else {
+                e = set_smem(simt_cached_kernel<float>, csmem);
+                if (e == cudaSuccess)
+                    e = launch_pdl(simt_cached_kernel<float>, grid, block, csmem, L.stream,
+                                   static_cast<const float*>(x), static_cast<const float*>(src),
+                                   static_cast<float*>(y), g.C, g.H, g.W, g.w, g.nh, g.nw, g.bands,
+                                   bpt, ntiles, tpb, G);
+            }
+            if (e != cudaSuccess)
+                return e;
+            note_launches(1);
+            return cudaGetLastError();
+        }
     }
     const size_t smem = ((mode == kCached ? 0 : (size_t)g.tsz) + (size_t)g.w * g.W) * 4;
     if (smem > kSimtSmemMax)
