@@ -82,8 +82,19 @@ def test_workspace_size_formula(lib):
     assert f(32, 4, 112, 112, 14, 1) == tc(4, 128)
     # 2 images of 112x112, w = 7: 64-window tiles of 4 bands, 8 tiles/channel
     assert f(2, 4, 112, 112, 7, 1) == tc(4, 32, 169)
-    # fp32, CUDA-core path: chunks of 8 bands per channel
+    # fp32, CUDA-core path, 4 <= w <= 14: tiles of whole bands (at most 64
+    # windows); all channels' tiles split into min(148, tiles) contiguous
+    # ranges; a channel spans at most 2 + (n - 2) // (fewest tiles of a
+    # range) of them (n tiles per channel, capped at n), one partial table
+    # slot each
     assert f(2, 3, 14, 28, 7, 0) == (65536 + 3 * 1 * 169) * 4
+    # training workload: 8 tiles per channel, 2048 tiles in ranges of 13 or 14
+    assert f(128, 256, 28, 28, 14, 0) == (65536 + 256 * 2 * 729) * 4
+    # 3 tiles per channel, 6 tiles, one per range: 3 slots
+    assert f(3, 2, 56, 56, 7, 0) == (65536 + 2 * 3 * 169) * 4
+    # w > 14: chunks of 8 bands per channel
+    assert f(2, 3, 40, 40, 20, 0) == (65536 + 3 * 1 * 1521) * 4
+    assert f(9, 1, 40, 40, 20, 0) == (65536 + 1 * 3 * 1521) * 4
     assert f(1, 1, 14, 15, 7, 1) == 0
 
 

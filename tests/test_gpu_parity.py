@@ -130,6 +130,40 @@ def test_backward_bf16_small(shape):
     check_bf16(to_np(dT), oracle.backward_dt(xr, gr, w), dt_bound(xr, gr, w), "dT")
 
 
+# CUDA-core table gradient as G = dY X^T and diagonal sums (4 <= w <= 14):
+# several tiles per channel with a ragged last tile, channels spread over
+# several blocks and blocks whose tile range crosses channel boundaries
+# (more tiles than the 148 blocks), a tile one window short of 64 (nw = 7),
+# one band per tile (nw = 64) and the bf16 inputs that take this path (rows
+# not 16-byte multiples), against the oracle.
+DTG_SHAPES = [(35, 2, 28, 28, 14, torch.float32), (3, 2, 56, 49, 7, torch.float32),
+              (20, 2, 30, 50, 10, torch.float32), (2, 2, 18, 576, 9, torch.float32),
+              (30, 2, 10, 15, 5, torch.bfloat16), (5, 3, 8, 8, 4, torch.float32),
+              (40, 60, 28, 28, 14, torch.float32), (4, 100, 56, 49, 7, torch.float32),
+              (30, 40, 10, 15, 5, torch.bfloat16)]
+
+
+@pytest.mark.parametrize("shape", DTG_SHAPES, ids=lambda s: "x".join(map(str, s[:5])) + str(s[5])[-4:])
+def test_cuda_core_table_gradient(shape):
+    B, C, H, W, w, dtype = shape
+    x = gen((B, C, H, W), 60, dtype)
+    dy = gen((B, C, H, W), 61, dtype)
+    T = gen((C, (2 * w - 1) ** 2), 62, dtype, 0.02)
+    dX, dT = wb.backward(x, T, dy, w)
+    torch.cuda.synchronize()
+    assert wb.wbmm_get_device_status() == 0
+    xr, gr = to_np(x), to_np(dy)
+    if dtype == torch.bfloat16:
+        check_bf16(to_np(dT), oracle.backward_dt(xr, gr, w), dt_bound(xr, gr, w), "dT")
+    else:
+        check_f32(to_np(dT), oracle.backward_dt(xr, gr, w),
+                  oracle.backward_dt(np.abs(xr), np.abs(gr), w), "dT")
+    # the fixed summation order gives the same bits on every call
+    dX2, dT2 = wb.backward(x, T, dy, w)
+    torch.cuda.synchronize()
+    assert torch.equal(dT, dT2)
+
+
 def test_dt_is_deterministic():
     B, C, H, W, w = 9, 3, 56, 56, 14
     x, dy = gen((B, C, H, W), 9), gen((B, C, H, W), 10)

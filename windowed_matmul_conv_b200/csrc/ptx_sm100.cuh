@@ -129,6 +129,13 @@ __device__ __forceinline__ void cp_async_4(uint32_t smem_dst, const void *gsrc)
                  : "memory");
 }
 
+// Global -> shared copy of 8 bytes, both addresses 8-byte aligned.
+__device__ __forceinline__ void cp_async_8(uint32_t smem_dst, const void *gsrc)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_dst), "l"(gsrc)
+                 : "memory");
+}
+
 __device__ __forceinline__ void cp_async_wait_all()
 {
     asm volatile("cp.async.wait_all;" ::: "memory");

@@ -4,6 +4,7 @@
 // mixing and the bounded-wait self-test.
 #include <cuda_bf16.h>
 
+#include <algorithm>
 #include <type_traits>
 
 #include <utility>
@@ -373,6 +374,243 @@ __global__ void simt_dt_kernel(const TIn* __restrict__ x, const TIn* __restrict_
     }
 }
 
+// Table gradient for 4 <= w <= 14 as G = dY X^T (positions x positions,
+// summed over windows) and diagonal sums: dT[dp, dq] adds G[(p, q),
+// (p - dp, q - dq)] over the positions where both are inside the window,
+// the same products the table-bin loop above forms.
+//
+// The tiles (whole bands, at most 64 windows) of all channels, channel by
+// channel, are split into gridDim.x contiguous ranges of equal size to
+// within one tile, one per block.  Per tile the dY and x windows sit in
+// shared memory as fp32 rows [window][position] (row stride DP = roundup(d,
+// 4*NCG); rows past the tile's windows are zero), two tiles deep so that the
+// next tile's copies overlap this tile's arithmetic; the copies go out in
+// units of V elements (V = 2 when w and W are even), every thread stepping
+// through the tile's rows and columns by a fixed stride without divisions.
+// Thread (ug, vg) accumulates G at rows 8ug .. 8ug+7 and columns k*CP +
+// 4vg .. k*CP + 4vg+3, k < NCG (CP = DP / NCG), over the windows in order:
+// 32*NCG fused multiply-adds per 2 + NCG 16-byte shared loads, and a warp
+// reads consecutive 16-byte words of the x rows.  Where its range leaves a channel, the block
+// puts G in shared memory; a warp per pair of window rows (p, p') sums the
+// 2w - 1 diagonals of that w x w block of G, lane by lane, then every bin
+// adds its (p, p - dp) sums in order of p into the partial table
+// [c][slot][tsz] (slot = block - first block of the channel).  The block of
+// slot 0 zeroes the slots the channel does not use, and the finaliser adds
+// all S slots in order.
+constexpr int kDtgSMs = 148;                // SMs of a B200
+constexpr int kDtgMaxCols = kCachedNT * 14; // window columns of a row, at most
+// Two column groups (8 x 8 thread tiles, 625 threads at w = 14) ran faster
+// than four (8 x 16, 325 threads): more warps cover the FMA latencies.
+constexpr int kDtgNCG = 2;                  // column groups of 4 per thread tile
+constexpr int kDtgMaxThreads = 640;         // thread tiles at w = 14, in whole warps
+
+template <typename TIn, int V>
+__global__ void __launch_bounds__(kDtgMaxThreads, 1)
+    simt_dtg_kernel(const TIn* __restrict__ x, const TIn* __restrict__ dy, float* __restrict__ part,
+                    int C, int H, int W, int w, int nh, int nw, long long bands, int bpt,
+                    int ntiles, int S)
+{
+    extern __shared__ __align__(16) float sgm[];
+    constexpr int NCG = kDtgNCG, TV = 4 * NCG;
+    const int d = w * w, DP = (d + TV - 1) / TV * TV, CP = DP / NCG;
+    const int UG = (d + 7) / 8, VG = CP / 4;
+    const int L = 2 * w - 1, tsz = L * L;
+    const int stage_floats = 2 * kCachedNT * DP;  // dY rows, then x rows
+    int* colmap = reinterpret_cast<int*>(sgm + 2 * stage_floats);
+    const long long G = gridDim.x, Ttot = (long long)C * ntiles;
+    const long long T0 = blockIdx.x * Ttot / G, T1 = (blockIdx.x + 1) * Ttot / G;
+    auto block_of = [&](long long f) { return ((f + 1) * G - 1) / Ttot; };
+    const int tid = threadIdx.x, nthr = blockDim.x;
+    const int lane = tid & 31, warp = tid >> 5, nwarps = nthr >> 5;
+    const int ug = tid / VG, vg = tid - (tid / VG) * VG;
+    const bool active = ug < UG;
+    // copy units of an image row: unit cu holds columns V*cu .. V*cu + V-1
+    // of window j, at offset j*DP + (position in the window row)
+    const int upr = nw * w / V;
+    for (int cu = tid; cu < upr; cu += nthr) {
+        const int col = cu * V, j = col / w;
+        colmap[cu] = j * DP + (col - j * w);
+    }
+    // this thread's first unit (row0, cu0) of a tile and its step: drow
+    // rows and dcu units (one more row when the unit index wraps)
+    const int row0 = tid / upr, cu0 = tid - (tid / upr) * upr;
+    const int drow = nthr / upr, dcu = nthr - (nthr / upr) * upr;
+    const int kb0 = row0 / w, r0 = row0 - (row0 / w) * w;
+    grid_dep_wait();
+    grid_dep_launch();
+    __syncthreads();
+    constexpr bool kAsync = std::is_same<TIn, float>::value;
+    // Tile f (flattened over channels) into stage st: asynchronous copies
+    // for fp32 (one commit group per tile), widened through registers for
+    // bf16.
+    auto load_tile = [&](long long f, int st) {
+        float* GS = sgm + (size_t)st * stage_floats;
+        float* XS = GS + kCachedNT * DP;
+        const int c = (int)(f / ntiles);
+        const long long g0 = (f - (long long)c * ntiles) * bpt;
+        const int nb = bands - g0 < bpt ? (int)(bands - g0) : bpt;
+        for (int e = tid; e < (kCachedNT - nb * nw) * DP; e += nthr) {
+            GS[nb * nw * DP + e] = 0.0f;
+            XS[nb * nw * DP + e] = 0.0f;
+        }
+        // band kb0 of the tile: image b, band i of that image
+        const long long gb = g0 + kb0;
+        long long b = gb / nh;
+        int i = (int)(gb - b * nh);
+        int kb = kb0, r = r0, cu = cu0;
+        while (kb < nb) {
+            const long long off = ((b * C + c) * H + (long long)i * w + r) * W + (long long)cu * V;
+            const int o = kb * nw * DP + r * w + colmap[cu];
+            if constexpr (kAsync) {
+                if constexpr (V == 2) {
+                    cp_async_8(smem_u32(GS + o), dy + off);
+                    cp_async_8(smem_u32(XS + o), x + off);
+                } else {
+                    cp_async_4(smem_u32(GS + o), dy + off);
+                    cp_async_4(smem_u32(XS + o), x + off);
+                }
+            } else {
+#pragma unroll
+                for (int v = 0; v < V; ++v) {
+                    GS[o + v] = to_f(dy[off + v]);
+                    XS[o + v] = to_f(x[off + v]);
+                }
+            }
+            cu += dcu;
+            int rinc = drow;
+            if (cu >= upr) {
+                cu -= upr;
+                ++rinc;
+            }
+            r += rinc;
+            while (r >= w) {
+                r -= w;
+                ++kb;
+                if (++i == nh) {
+                    i = 0;
+                    ++b;
+                }
+            }
+        }
+        if constexpr (kAsync)
+            cp_async_commit();
+    };
+    float acc[8][TV];
+#pragma unroll
+    for (int a = 0; a < 8; ++a)
+#pragma unroll
+        for (int b = 0; b < TV; ++b)
+            acc[a][b] = 0.0f;
+    int st = 0;
+    if (T0 < T1)
+        load_tile(T0, 0);
+    for (long long f = T0; f < T1; ++f) {
+        const int c = (int)(f / ntiles);
+        const bool same_next = f + 1 < T1 && (f + 1) / ntiles == c;
+        // stage st ^ 1 was last read by the previous tile, before the barrier
+        // that closed its iteration
+        if (same_next)
+            load_tile(f + 1, st ^ 1);
+        if constexpr (kAsync) {
+            if (same_next)
+                cp_async_wait_group<1>();
+            else
+                cp_async_wait_group<0>();
+        }
+        __syncthreads();
+        if (active) {
+            const float* ap = sgm + (size_t)st * stage_floats + 8 * ug;
+            const float* bp = sgm + (size_t)st * stage_floats + kCachedNT * DP + 4 * vg;
+#pragma unroll 2
+            for (int n = 0; n < kCachedNT; ++n) {
+                const float4 a0 = *reinterpret_cast<const float4*>(ap + n * DP);
+                const float4 a1 = *reinterpret_cast<const float4*>(ap + n * DP + 4);
+                float bv[TV];
+#pragma unroll
+                for (int k = 0; k < NCG; ++k) {
+                    const float4 bk = *reinterpret_cast<const float4*>(bp + n * DP + k * CP);
+                    bv[4 * k] = bk.x;
+                    bv[4 * k + 1] = bk.y;
+                    bv[4 * k + 2] = bk.z;
+                    bv[4 * k + 3] = bk.w;
+                }
+                const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+#pragma unroll
+                for (int a = 0; a < 8; ++a)
+#pragma unroll
+                    for (int b = 0; b < TV; ++b)
+                        acc[a][b] = __fmaf_rn(av[a], bv[b], acc[a][b]);
+            }
+        }
+        __syncthreads();
+        if (same_next) {
+            st ^= 1;
+            continue;
+        }
+        // ------------------------------------------- channel c's partial
+        // G[u][v] to shared memory (the operand stages are dead); rows u >= d
+        // are not written, columns v >= d are written but never read.  The
+        // diagonal sums R[p][p'][dq + w - 1] follow G.
+        float* GM = sgm;
+        float* RS = sgm + (size_t)d * DP;
+        if (active) {
+#pragma unroll
+            for (int a = 0; a < 8; ++a) {
+                const int u = 8 * ug + a;
+                if (u < d) {
+#pragma unroll
+                    for (int k = 0; k < NCG; ++k)
+                        *reinterpret_cast<float4*>(GM + u * DP + k * CP + 4 * vg) =
+                            make_float4(acc[a][4 * k], acc[a][4 * k + 1], acc[a][4 * k + 2],
+                                        acc[a][4 * k + 3]);
+                }
+            }
+        }
+#pragma unroll
+        for (int a = 0; a < 8; ++a)
+#pragma unroll
+            for (int b = 0; b < TV; ++b)
+                acc[a][b] = 0.0f;
+        __syncthreads();
+        // block (p, p') of G: rows p*w + q, columns p'*w + q'; lane l sums
+        // its diagonal q - q' = l - (w - 1) in order of q
+        for (int pr = warp; pr < d; pr += nwarps) {
+            const int p = pr / w, p2 = pr - (pr / w) * w;
+            if (lane < L) {
+                const int dq = lane - (w - 1);
+                const int q0 = dq > 0 ? dq : 0, q1 = dq > 0 ? w : w + dq;
+                const float* gp = GM + (p * w + q0) * DP + p2 * w + (q0 - dq);
+                float sum = 0.0f;
+                for (int q = q0; q < q1; ++q, gp += DP + 1)
+                    sum += *gp;
+                RS[pr * L + lane] = sum;
+            }
+        }
+        __syncthreads();
+        const long long first = block_of((long long)c * ntiles);
+        const int slot = (int)(blockIdx.x - first);
+        float* out = part + ((long long)c * S + slot) * tsz;
+        for (int bin = tid; bin < tsz; bin += nthr) {
+            const int dpi = bin / L, dqi = bin - (bin / L) * L;
+            const int dp = dpi - (w - 1);
+            const int p0 = dp > 0 ? dp : 0, p1 = dp > 0 ? w : w + dp;
+            float sum = 0.0f;
+            for (int p = p0; p < p1; ++p)
+                sum += RS[(p * w + p - dp) * L + dqi];
+            out[bin] = sum;
+        }
+        if (slot == 0) {
+            const int used = (int)(block_of((long long)c * ntiles + ntiles - 1) - first) + 1;
+            for (int e = used * tsz + tid; e < S * tsz; e += nthr)
+                part[(long long)c * S * tsz + e] = 0.0f;
+        }
+        __syncthreads();        // RS read before the next tile's copies land
+        if (f + 1 < T1)
+            load_tile(f + 1, 0);
+        st = 0;
+    }
+}
+
 // Fixed-order sum of the partial tables.
 __global__ void dt_finalize_kernel(const float* __restrict__ part, float* __restrict__ dT, int C,
                                    int tsz, int chunks)
@@ -607,8 +845,66 @@ constexpr size_t kSimtSmemMax = 200 * 1024;
 
 }  // namespace
 
+namespace {
+
+// one thread per 8 x 4*kDtgNCG block of G, in whole warps
+int dtg_threads(const Geom& g)
+{
+    const int d = g.w * g.w, TV = 4 * kDtgNCG;
+    return ((d + 7) / 8 * ((d + TV - 1) / TV) + 31) / 32 * 32;
+}
+
+size_t dtg_smem(const Geom& g)
+{
+    const int d = g.w * g.w, DP = (d + 4 * kDtgNCG - 1) / (4 * kDtgNCG) * (4 * kDtgNCG);
+    // two stages of dY and x rows (G and the diagonal row sums fit in them),
+    // then the column map
+    return (size_t)4 * kCachedNT * DP * 4 + (size_t)kDtgMaxCols * 4;
+}
+
+// The register-tiled table gradient's plan: whole bands per tile, tiles per
+// channel, blocks, and partial-table slots per channel.  A channel's tiles
+// span at most 2 + (ntiles - 2) / (fewest tiles of a block) blocks: every
+// block strictly inside the span covers that many of the channel's tiles.
+// Returns false when the shape takes the table-bin kernel instead.
+struct DtgPlan {
+    int bpt, ntiles, grid, slots;
+};
+
+bool dtg_plan(const Geom& g, DtgPlan& pl)
+{
+    if (g.w < 4 || g.w > 14 || g.nw < 1 || g.nw > kCachedNT || g.bands < 1 || g.C < 1 ||
+        g.nw * g.w > kDtgMaxCols)
+        return false;
+    pl.bpt = kCachedNT / g.nw;
+    const long long nt = (g.bands + pl.bpt - 1) / pl.bpt;
+    const long long total = nt * g.C;
+    if (nt > (1 << 30) || total > (1ll << 40))
+        return false;
+    pl.ntiles = (int)nt;
+    // blocks resident per SM, by shared memory (233472 bytes per SM, 1 KB
+    // reserved per block), threads and registers (at most the launch
+    // bound's share of 65536 per thread)
+    const int threads = dtg_threads(g);
+    const int regs = 65536 / kDtgMaxThreads / 8 * 8;
+    int bps = (int)(233472 / (dtg_smem(g) + 1024));
+    bps = std::min(bps, 2048 / threads);
+    bps = std::max(1, std::min(bps, 65536 / (threads * regs)));
+    const long long want = (long long)kDtgSMs * bps;
+    pl.grid = (int)(total < want ? total : want);
+    const long long fewest = total / pl.grid;
+    const long long span = nt == 1 ? 1 : 2 + (nt - 2) / fewest;
+    pl.slots = (int)(span < nt ? span : nt);
+    return true;
+}
+
+}  // namespace
+
 int simt_dt_chunks(const Geom& g)
 {
+    DtgPlan pl;
+    if (dtg_plan(g, pl))
+        return pl.slots;
     return (int)((g.bands + kSimtChunkBands - 1) / kSimtChunkBands);
 }
 
@@ -744,6 +1040,35 @@ cudaError_t simt_fwd_launch(const Geom& g, AMode mode, bool is_bf16, const void*
 cudaError_t simt_dt_launch(const Geom& g, bool is_bf16, const void* x, const void* dy,
                            float* partials, const Launch& L)
 {
+    DtgPlan pl;
+    if (dtg_plan(g, pl)) {
+        const int threads = dtg_threads(g);
+        const size_t smem = dtg_smem(g);
+        const dim3 grid((unsigned)pl.grid), block(threads);
+        // two-element copies need even w and W and 8-byte aligned fp32 rows
+        const bool pairs = g.w % 2 == 0 && g.W % 2 == 0 &&
+                           ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(dy)) & 7) == 0;
+        cudaError_t e;
+        if (is_bf16) {
+            using E = __nv_bfloat16;
+            e = set_smem(simt_dtg_kernel<E, 1>, smem);
+            if (e == cudaSuccess)
+                e = launch_pdl(simt_dtg_kernel<E, 1>, grid, block, smem, L.stream,
+                               static_cast<const E*>(x), static_cast<const E*>(dy), partials, g.C,
+                               g.H, g.W, g.w, g.nh, g.nw, g.bands, pl.bpt, pl.ntiles, pl.slots);
+        } else {
+            auto kern = pairs ? simt_dtg_kernel<float, 2> : simt_dtg_kernel<float, 1>;
+            e = set_smem(kern, smem);
+            if (e == cudaSuccess)
+                e = launch_pdl(kern, grid, block, smem, L.stream, static_cast<const float*>(x),
+                               static_cast<const float*>(dy), partials, g.C, g.H, g.W, g.w, g.nh,
+                               g.nw, g.bands, pl.bpt, pl.ntiles, pl.slots);
+        }
+        if (e != cudaSuccess)
+            return e;
+        note_launches(1);
+        return cudaGetLastError();
+    }
     const size_t smem = (size_t)2 * g.w * g.W * 4;
     // each thread owns up to kSimtMaxBinsPerThread table entries: 256 threads
     // cover w <= 32, 1024 threads every w the library accepts (<= 64)
