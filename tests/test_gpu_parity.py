@@ -346,10 +346,13 @@ def test_reparam_merge_argument_errors():
     assert wb.wbmm_launch_count() == before
 
 
-# (B, C, H, W, w): fused work units of one tile holding several planes
-# (56x56, 48x48 at w=16) and of one plane spanning several tiles (112x56 at
-# w=7, 224x224)
-FUSED_SHAPES = [(3, 2, 56, 56, 14), (2, 3, 112, 56, 7), (2, 2, 48, 48, 16), (2, 3, 224, 224, 14)]
+# (B, C, H, W, w): tiles holding several whole planes (56x56, 42x56 with the
+# tile cut to 30 bands, 70x112 with 15 and a partial last tile), planes of
+# two tiles (224x224, 168x168 with tiles cut to 6 bands) and of three
+# (336x224), one plane per tile (112x56 at w = 7), and w = 16 (the older
+# fused kernel)
+FUSED_SHAPES = [(3, 2, 56, 56, 14), (2, 3, 112, 56, 7), (2, 2, 48, 48, 16), (2, 3, 224, 224, 14),
+                (2, 2, 42, 56, 14), (2, 2, 168, 168, 14), (1, 2, 336, 224, 14), (4, 2, 70, 112, 14)]
 
 
 @pytest.mark.parametrize("shape", FUSED_SHAPES, ids=lambda s: "x".join(map(str, s)))
@@ -377,13 +380,13 @@ def test_fused_cached_dw3x3_matches_two_calls(shape):
 
 
 def test_fused_cached_dw3x3_unsupported_shapes():
-    # window rows per tile (16) and per image (3) do not divide each other
-    x = gen((2, 2, 42, 56), 24)
-    M = wb.cache_matrices(gen((2, 729), 25, scale=0.02), 14)
+    # image rows that are not whole 16-byte vectors (W = 12)
+    x = gen((2, 2, 12, 12), 24)
+    M = wb.cache_matrices(gen((2, 49), 25, scale=0.02), 4)
     K = gen((2, 1, 3, 3), 26)
     before = wb.wbmm_launch_count()
     with pytest.raises(wb.WbmmError) as e:
-        wb.forward_cached(x, M, 14, dw=K)
+        wb.forward_cached(x, M, 4, dw=K)
     assert e.value.status == 5
     # fp32 maps
     xf = gen((1, 2, 14, 14), 27, torch.float32)
@@ -522,6 +525,11 @@ def test_full_size_cached_dw_sampled():
     # the forward row bound
     zb = oracle.dw3x3(forward_rowbound(xs, Ts, wl.w), np.abs(Ks))
     check_bf16(to_np(z[bs][:, cs]), zref, zb, "hires z")
+    # the fused launch gives the two calls' bits at full size
+    zf = wb.forward_cached(x, M, wl.w, dw=K)
+    torch.cuda.synchronize()
+    assert wb.wbmm_get_device_status() == 0
+    assert torch.equal(zf, z)
 
 
 def test_full_size_fp32_training_step_sampled():

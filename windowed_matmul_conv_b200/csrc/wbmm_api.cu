@@ -397,8 +397,8 @@ wbmm_status wbmm_forward_cached(const void* x, const void* M, const void* dw3x3,
     if ((st = make_launch(stream, &L)) != WBMM_OK)
         return st;
     const bool fused = dw3x3 != nullptr;
-    if (dt == WBMM_BF16 && !fused && tc_cached_supported(g)) {
-        st = from_cuda(tc_cached_launch(g, x, M, out, L));
+    if (dt == WBMM_BF16 && tc_cached_supported(g, fused)) {
+        st = from_cuda(tc_cached_launch(g, x, M, dw3x3, out, L));
         if (st == WBMM_OK)
             t_last_path = 1;
         return st;

@@ -72,9 +72,9 @@ cudaError_t tc_big_launch(const Geom& g, AMode mode, const void* x, const void* 
                           const Launch& L);
 
 // tcgen05 forward with a cached [C][d][d] matrix, windows as the MMA's M
-// dimension (no fused 3x3).
-bool tc_cached_supported(const Geom& g);
-cudaError_t tc_cached_launch(const Geom& g, const void* x, const void* M, void* y,
+// dimension; with dw (fuse) the epilogue applies the 3x3 mixing and y is z.
+bool tc_cached_supported(const Geom& g, bool fuse);
+cudaError_t tc_cached_launch(const Geom& g, const void* x, const void* M, const void* dw, void* y,
                              const Launch& L);
 
 // tcgen05 table gradient: one contiguous tile range per CTA.  The workspace

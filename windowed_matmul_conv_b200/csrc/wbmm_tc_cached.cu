@@ -27,6 +27,14 @@
 //                tile of each channel, whose completion implies that every
 //                MMA reading the previous B has finished
 //
+// Fused 3x3 mixing (FUSE, the inter-block depthwise step that follows the
+// cached forward): the CTA ranges are whole image planes; after each tile's
+// drain the transform and epilogue warps (16 workers) apply the 3x3 to the
+// bf16 y rows in the staging buffer, carrying the two rows at a tile edge
+// inside a plane to the next tile, and store z from registers; the storer
+// idles and y never reaches HBM.  Bit-identical to the cached forward
+// followed by the standalone 3x3 kernel.
+//
 // TMEM: A stages at columns 0 and 128; the accumulator at 256, in two halves
 // of output positions (256 and 384) when there are more than 128 of them.
 // Every wait is bounded; a wait that runs out raises the CTA's abort flag and
@@ -36,6 +44,7 @@
 
 #include <type_traits>
 
+#include "dw_common.cuh"
 #include "ptx_sm100.cuh"
 #include "tc_common.cuh"
 #include "wbmm_internal.h"
@@ -78,6 +87,8 @@ constexpr int kCXformWarps = 8;
 constexpr int kCEpiWarp0 = kCXformWarp0 + kCXformWarps;
 constexpr int kCEpiWarps = 8;
 constexpr int kCThreads = (kCEpiWarp0 + kCEpiWarps) * 32;
+// fused 3x3: the transform and epilogue warps share each tile's stencil
+constexpr int kFuseWorkers = kCXformWarps + kCEpiWarps;
 constexpr int kCTileWindows = 128;
 
 struct TcCachedParams {
@@ -85,12 +96,14 @@ struct TcCachedParams {
     TmapBytes map_y;        // output planes, one box = a tile (use_tmap)
     const uint16_t* x;
     const uint16_t* M;      // [C][d][d] bf16, row u = p*w+q
-    uint16_t* y;
+    uint16_t* y;            // y, or z = 3x3(y) when fused
+    const uint16_t* dw;     // fused: [C][3][3] bf16 weights
     int C, H, W, nh, nw;
     int bpt, sb, tpc, bands, items, R;
+    int unit;               // tiles per unit of the CTA ranges (fused: whole planes)
     uint32_t sub_bytes;
     int use_tmap, kimg_sub;
-    uint32_t off_b, off_out, off_raw, off_woff, off_bar;
+    uint32_t off_b, off_out, off_raw, off_bar, off_halo;
     unsigned long long budget;
     int* status;
 };
@@ -206,7 +219,134 @@ __device__ __forceinline__ uint32_t cbf16x2_rn(uint32_t lo, uint32_t hi)
     return *reinterpret_cast<const uint32_t*>(&v);
 }
 
+// Fused 3x3 mixing of one tile, run by the transform and epilogue warps
+// once the tile's bf16 y rows are in the output buffer (row R = k*w + r of
+// the tile's bands, W elements, i.e. image rows in order).  Rows R = -2, -1
+// are the previous tile's last two rows (a halo buffer), valid when the tile
+// starts inside a plane; that tile's last output row waits for this tile's
+// first row and is made here (R = -1).  Likewise this tile's last row is left
+// to the next tile when the plane continues.  Worker k of nworkers takes a
+// contiguous range of output rows; lane = 16-byte vector of a row.  The
+// worker streams the input rows once, in order: input row i adds its taps
+// of kernel row a = 0 to output i+1, a = 1 to output i and a = 2 to output
+// i-1, so every output receives the standalone kernel's fp32 fused
+// multiply-adds in the same (a, e) order (dw3x3_pairs8).  Taps that would
+// read across a plane edge are left out instead of multiplying zeros: an
+// accumulator that starts at +0 never holds -0, so adding a zero product
+// never changes it and the bits are the same.  z goes to HBM straight from
+// registers.
 template <int WS>
+__device__ __forceinline__ void fused_dw_rows(const TcCachedParams& P, const BandTile& t,
+                                              const uint16_t* ybuf, const uint16_t* halo,
+                                              int worker, int nworkers, int lane)
+{
+    const int W = P.W, nv = W >> 3, H = P.nh * WS;
+    const int nbw = t.nb * WS;
+    const int pr0 = (t.band0 % P.nh) * WS;          // plane row of the tile's row 0
+    const bool next_cont = (t.band0 + t.nb) % P.nh != 0;
+    const int r_lo = pr0 != 0 ? -1 : 0, r_hi = next_cont ? nbw - 1 : nbw;
+    const int cnt = r_hi - r_lo;
+    const int rs = r_lo + worker * cnt / nworkers, re = r_lo + (worker + 1) * cnt / nworkers;
+    if (rs >= re)
+        return;
+    float k[9];
+#pragma unroll
+    for (int m = 0; m < 9; ++m)
+        k[m] = __bfloat162float(__ushort_as_bfloat16(P.dw[(long long)t.c * 9 + m]));
+    // plane row and image of input row rs - 1 (plane row -1: the row above
+    // the tile when the tile starts a plane, which belongs to no output)
+    int p1, b1;
+    if (rs - 1 < 0) {
+        p1 = pr0 + rs - 1;
+        b1 = t.band0 / P.nh;
+    } else {
+        const int gb = t.band0 + (rs - 1) / WS;
+        b1 = gb / P.nh;
+        p1 = (gb - b1 * P.nh) * WS + (rs - 1) % WS;
+    }
+    const long long plane_step = (long long)P.C * H * W;   // next image, same channel
+    for (int v = lane; v < nv; v += 32) {
+        int pi = p1;                                // plane row of input row i
+        // z addresses of rows i (zc) and i - 1 (zo); row -1 of an image is
+        // the address one row before its row 0
+        uint16_t* zc = P.y + (((long long)b1 * P.C + t.c) * H + p1) * W + 8 * v;
+        uint16_t* zo = zc;
+        const uint16_t* yrow = (rs - 1 >= 0 ? ybuf + (size_t)(rs - 1) * W
+                                            : halo + (size_t)(rs + 1) * W) + 8 * v;
+        // Input row i: X holds output i-1 (kernel row 2, then stored), Y
+        // output i (kernel row 1), Z output i+1 (started here, kernel row 0).
+        float X[8], Y[8], Z[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            X[j] = Y[j] = 0.0f;
+        for (int i = rs - 1; i <= re; ++i) {
+            const bool c_up = i + 1 >= rs && i + 1 < re && pi >= 0 && pi + 1 < H;
+            const bool c_mid = i >= rs && i < re;
+            const bool c_dn = i - 1 >= rs && i - 1 < re && pi > 0;
+            float u[10];
+            if (c_up || c_mid || c_dn) {
+                const uint4 q = *reinterpret_cast<const uint4*>(yrow);
+                u[0] = v > 0 ? __uint_as_float((uint32_t)yrow[-1] << 16) : 0.0f;
+                u[9] = v + 1 < nv ? __uint_as_float((uint32_t)yrow[8] << 16) : 0.0f;
+                const uint32_t w4[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    u[1 + 2 * j] = __uint_as_float(w4[j] << 16);
+                    u[2 + 2 * j] = __uint_as_float(w4[j] & 0xFFFF0000u);
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                Z[j] = 0.0f;
+            if (c_up) {
+#pragma unroll
+                for (int e = 0; e < 3; ++e)
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        Z[j] = __fmaf_rn(k[e], u[j + e], Z[j]);
+            }
+            if (c_mid) {
+#pragma unroll
+                for (int e = 0; e < 3; ++e)
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        Y[j] = __fmaf_rn(k[3 + e], u[j + e], Y[j]);
+            }
+            if (c_dn) {
+#pragma unroll
+                for (int e = 0; e < 3; ++e)
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        X[j] = __fmaf_rn(k[6 + e], u[j + e], X[j]);
+            }
+            if (i - 1 >= rs && i - 1 < re) {
+                uint32_t packed[4];
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    const __nv_bfloat162 h2 = __floats2bfloat162_rn(X[2 * m], X[2 * m + 1]);
+                    packed[m] = *reinterpret_cast<const uint32_t*>(&h2);
+                }
+                *reinterpret_cast<uint4*>(zo) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+            }
+            // advance to row i + 1: the halo rows are followed by the tile's
+            // row 0, and the next plane starts one image later
+            yrow = i == -1 ? ybuf + 8 * v : yrow + W;
+            zo = zc;
+            zc += W;
+            if (++pi == H) {
+                pi = 0;
+                zc += plane_step - (long long)H * W;
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                X[j] = Y[j];
+                Y[j] = Z[j];
+            }
+        }
+    }
+}
+
+template <int WS, bool FUSE>
 __global__ void __launch_bounds__(kCThreads, 1)
     wbmm_tc_cached_kernel(const __grid_constant__ TcCachedParams P)
 {
@@ -216,14 +356,17 @@ __global__ void __launch_bounds__(kCThreads, 1)
     uint8_t* b_base = smem + P.off_b;
     uint8_t* out_base = smem + P.off_out;
     uint8_t* raw_base = smem + P.off_raw;
-    int* woff = reinterpret_cast<int*>(smem + P.off_woff);
+    // offset of window m of a band-layout buffer (band k = m / nw, column j)
+    auto woff = [&](int m) { return (m / P.nw) * WS * P.W + (m % P.nw) * WS; };
     CachedBars& S = *reinterpret_cast<CachedBars*>(smem + P.off_bar);
     volatile int* abort = &S.abort;
     const int R = P.R;
 
-    const int qn = P.items / (int)gridDim.x, rem = P.items % (int)gridDim.x;
-    const int it0 = (int)blockIdx.x * qn + ((int)blockIdx.x < rem ? (int)blockIdx.x : rem);
-    const int n_it = qn + ((int)blockIdx.x < rem ? 1 : 0);
+    // a contiguous, balanced range of units (P.unit tiles each) per CTA
+    const int units = P.items / P.unit;
+    const int qn = units / (int)gridDim.x, rem = units % (int)gridDim.x;
+    const int it0 = ((int)blockIdx.x * qn + ((int)blockIdx.x < rem ? (int)blockIdx.x : rem)) * P.unit;
+    const int n_it = (qn + ((int)blockIdx.x < rem ? 1 : 0)) * P.unit;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kCRing; ++i) {
@@ -245,10 +388,6 @@ __global__ void __launch_bounds__(kCThreads, 1)
         S.abort = 0;
         fence_mbar_init();
     }
-    for (int n = threadIdx.x; n < kCTileWindows; n += kCThreads) {
-        const int k = n / P.nw, j = n - k * P.nw;
-        woff[n] = k * WS * P.W + j * WS;
-    }
     if (warp == 1) {
         tmem_alloc(&S.tmem_slot, 512);
         tmem_relinquish();
@@ -257,6 +396,30 @@ __global__ void __launch_bounds__(kCThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = S.tmem_slot;
+    // Fused 3x3 of tile sq (FUSE): every transform and epilogue thread calls
+    // this once per tile, in tile order, whatever its wait results.  The
+    // first barrier is reached by the epilogue warps after draining tile sq
+    // and by the transform warps after writing the A operand of tile sq + 1;
+    // the stencil reads the halo buffer (sq + 1) & 1, and the epilogue threads
+    // keep the tile's last two rows in buffer sq & 1 for the next tile.
+    auto fused_stage = [&](int sq, int worker, bool epi) {
+        const BandTile ft = cached_tile(P, it0 + sq);
+        const uint16_t* ybuf = reinterpret_cast<const uint16_t*>(out_base);
+        uint16_t* halo = reinterpret_cast<uint16_t*>(smem + P.off_halo);
+        const size_t hsz = 2 * (size_t)P.W;
+        named_bar_sync(2, kFuseWorkers * 32);       // y rows of tile sq written
+        if (!*abort)
+            fused_dw_rows<WS>(P, ft, ybuf, halo + ((sq + 1) & 1) * hsz, worker, kFuseWorkers,
+                              lane);
+        if (epi && (ft.band0 + ft.nb) % P.nh != 0) {
+            const int nvec2 = 2 * (P.W >> 3);
+            const uint4* src = reinterpret_cast<const uint4*>(ybuf + (size_t)(ft.nb * WS - 2) * P.W);
+            uint4* dst = reinterpret_cast<uint4*>(halo + (sq & 1) * hsz);
+            for (int i = (int)threadIdx.x - kCEpiWarp0 * 32; i < nvec2; i += kCEpiWarps * 32)
+                dst[i] = src[i];
+        }
+        named_bar_sync(2, kFuseWorkers * 32);       // the buffer and halo rows are read
+    };
     // Everything above overlaps the previous kernel's tail; tensors are read
     // and written only after it has completed.
     grid_dep_wait();
@@ -371,7 +534,8 @@ __global__ void __launch_bounds__(kCThreads, 1)
         }
     } else if (warp == 2) {
         // ------------------------------------------------------ storer
-        for (int seq = 0; seq < n_it; ++seq) {
+        // (fused: the stencil workers store z themselves)
+        for (int seq = 0; seq < (FUSE ? 0 : n_it); ++seq) {
             bool ok = !*abort;
             ok = ok && mbar_wait(&S.out_full, seq & 1, abort, P.budget, P.status);
             ok = __all_sync(0xffffffffu, ok);
@@ -428,7 +592,7 @@ __global__ void __launch_bounds__(kCThreads, 1)
                 const int h = n < h0win ? 0 : 1;
                 const uint16_t* raw = reinterpret_cast<const uint16_t*>(
                     raw_base + (size_t)(h ? s1 : s0) * P.sub_bytes);
-                const uint16_t* src0 = raw + (valid ? woff[h ? n - h0win : n] : 0);
+                const uint16_t* src0 = raw + (valid ? woff(h ? n - h0win : n) : 0);
                 const uint32_t acol = tmem + lanebase + (uint32_t)(st * 128);
 #pragma unroll 2
                 for (int r = r_lo; r < r_hi; ++r) {
@@ -466,6 +630,14 @@ __global__ void __launch_bounds__(kCThreads, 1)
                 mbar_arrive(&S.raw_empty[s1]);
                 mbar_arrive(&S.a_full[st]);
             }
+            if constexpr (FUSE) {
+                if (seq >= 1)
+                    fused_stage(seq - 1, warp - kCXformWarp0, false);
+            }
+        }
+        if constexpr (FUSE) {
+            if (n_it >= 1)
+                fused_stage(n_it - 1, warp - kCXformWarp0, false);
         }
     } else {
         // ------------------------------------------------------ epilogue
@@ -490,10 +662,10 @@ __global__ void __launch_bounds__(kCThreads, 1)
             const BandTile t = cached_tile(P, it0 + seq);
             const int nwin = t.nb * P.nw;
             bool ok = !*abort;
-            if (seq >= 1)
+            if (!FUSE && seq >= 1)
                 ok = ok && mbar_wait(&S.out_empty, (seq - 1) & 1, abort, P.budget, P.status);
             const bool valid = n < nwin;
-            uint16_t* o0 = reinterpret_cast<uint16_t*>(out_base) + (valid ? woff[n] : 0);
+            uint16_t* o0 = reinterpret_cast<uint16_t*>(out_base) + (valid ? woff(n) : 0);
             // output positions [E0, E1) from the accumulator columns at lbase
             // (position E0 at column 0); warp half hf takes every other
             // 32-column load.  Positions are compile-time constants, so the
@@ -562,12 +734,15 @@ __global__ void __launch_bounds__(kCThreads, 1)
             if (ok && lane == 0) {
                 if constexpr (!F::NSPLIT)
                     mbar_arrive(&S.acc_empty[0]);
-                mbar_arrive(&S.out_full);
+                if constexpr (!FUSE)
+                    mbar_arrive(&S.out_full);
             }
             // the channel's last tile is done: every MMA that read B has
             // completed (acc_full), so B can take the next channel's matrix
             if (seq + 1 < n_it && cached_tile(P, it0 + seq + 1).c != t.c)
                 build_for(t.c + 1);
+            if constexpr (FUSE)
+                fused_stage(seq, kCXformWarps + warp - kCEpiWarp0, true);
         }
     }
 
@@ -589,17 +764,32 @@ constexpr uint32_t kMinSmem = 120 * 1024;
 inline uint32_t align_up(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
 
 struct CachedLayout {
-    uint32_t off_b, off_out, off_raw, off_woff, off_bar, total, sub_bytes;
-    int R, bpt, sb;
+    uint32_t off_b, off_out, off_raw, off_bar, off_halo, total, sub_bytes;
+    int R, bpt, sb, unit;
 };
 
+// fuse: the 3x3 runs in the epilogue; it needs whole 16-byte vectors per
+// row and tiles that hold whole planes or planes of whole tiles (the CTA
+// ranges are then whole planes), plus two halo rows of shared memory.
 template <int WS>
-bool cached_layout(const Geom& g, CachedLayout& L)
+bool cached_layout(const Geom& g, CachedLayout& L, bool fuse)
 {
     using F = CachedCfg<WS>;
     if (g.nw < 1 || g.nw > kCTileWindows)
         return false;
     L.bpt = kCTileWindows / g.nw;
+    L.unit = 1;
+    if (fuse) {
+        if (g.W % 8 != 0)
+            return false;
+        if (L.bpt >= g.nh) {
+            L.bpt = L.bpt / g.nh * g.nh;            // whole planes per tile
+        } else {
+            while (g.nh % L.bpt != 0)               // planes of whole tiles
+                --L.bpt;
+            L.unit = g.nh / L.bpt;
+        }
+    }
     L.sb = (L.bpt + 1) / 2;
     L.sub_bytes = align_up((uint32_t)L.sb * WS * g.W * 2, 128);
     uint32_t off = 0;
@@ -607,37 +797,46 @@ bool cached_layout(const Geom& g, CachedLayout& L)
     off += F::B_BYTES;
     L.off_out = align_up(off, 128);
     off = L.off_out + F::OUT_BYTES;
-    L.off_woff = align_up(off, 16);
-    off = L.off_woff + kCTileWindows * 4;
     L.off_bar = align_up(off, 16);
     off = L.off_bar + sizeof(CachedBars);
+    L.off_halo = align_up(off, 16);
+    if (fuse)
+        off = L.off_halo + 2u * 2u * (uint32_t)g.W * 2u;     // two halo buffers of two rows
     L.off_raw = align_up(off, 128);
-    const uint32_t avail = kSmemMax - 1024 > L.off_raw ? kSmemMax - 1024 - L.off_raw : 0;
+    // the fused layout is not rounded up to 1 KB, which keeps a third ring
+    // slot at 224 x 224
+    const uint32_t reserve = fuse ? 0u : 1024u;
+    const uint32_t avail = kSmemMax - reserve > L.off_raw ? kSmemMax - reserve - L.off_raw : 0;
     int R = (int)(avail / L.sub_bytes);
     if (R > kCRing)
         R = kCRing;
     L.R = R;
     if (R < 2)
         return false;
-    L.total = align_up(L.off_raw + (uint32_t)R * L.sub_bytes, 1024);
+    L.total = align_up(L.off_raw + (uint32_t)R * L.sub_bytes, fuse ? 128u : 1024u);
     if (L.total < kMinSmem)
         L.total = kMinSmem;
     return L.total <= kSmemMax;
 }
 
 template <int WS>
-cudaError_t cached_launch_ws(const Geom& g, const void* x, const void* M, void* y, const Launch& L)
+cudaError_t cached_launch_ws(const Geom& g, const void* x, const void* M, const void* dw, void* y,
+                             const Launch& L)
 {
+    const bool fuse = dw != nullptr;
     CachedLayout lay;
-    if (!cached_layout<WS>(g, lay))
+    if (!cached_layout<WS>(g, lay, fuse))
         return cudaErrorInvalidConfiguration;
     static int configured[64] = {0};
     int dev = 0;
     cudaGetDevice(&dev);
     if (!configured[dev & 63]) {
-        cudaError_t e = cudaFuncSetAttribute(wbmm_tc_cached_kernel<WS>,
+        cudaError_t e = cudaFuncSetAttribute(wbmm_tc_cached_kernel<WS, false>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)kSmemMax);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(wbmm_tc_cached_kernel<WS, true>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemMax);
         if (e != cudaSuccess)
             return e;
         configured[dev & 63] = 1;
@@ -646,9 +845,11 @@ cudaError_t cached_launch_ws(const Geom& g, const void* x, const void* M, void* 
     P.x = static_cast<const uint16_t*>(x);
     P.M = static_cast<const uint16_t*>(M);
     P.y = static_cast<uint16_t*>(y);
+    P.dw = static_cast<const uint16_t*>(dw);
     P.C = g.C; P.H = g.H; P.W = g.W; P.nh = g.nh; P.nw = g.nw;
     P.bpt = lay.bpt;
     P.sb = lay.sb;
+    P.unit = lay.unit;
     P.bands = (int)g.bands;
     P.tpc = (P.bands + P.bpt - 1) / P.bpt;
     P.items = g.C * P.tpc;
@@ -664,16 +865,18 @@ cudaError_t cached_launch_ws(const Geom& g, const void* x, const void* M, void* 
         }
     }
     P.off_b = lay.off_b; P.off_out = lay.off_out; P.off_raw = lay.off_raw;
-    P.off_woff = lay.off_woff; P.off_bar = lay.off_bar;
+    P.off_bar = lay.off_bar; P.off_halo = lay.off_halo;
     P.budget = L.budget;
     P.status = L.status;
     int grid = L.num_sms;
-    if (grid > P.items)
-        grid = P.items;
+    if (grid > P.items / P.unit)
+        grid = P.items / P.unit;
     if (grid < 1)
         return cudaSuccess;
-    cudaError_t e = launch_pdl(wbmm_tc_cached_kernel<WS>, dim3(grid), dim3(kCThreads), lay.total,
-                               L.stream, P);
+    cudaError_t e = fuse ? launch_pdl(wbmm_tc_cached_kernel<WS, true>, dim3(grid), dim3(kCThreads),
+                                      lay.total, L.stream, P)
+                         : launch_pdl(wbmm_tc_cached_kernel<WS, false>, dim3(grid),
+                                      dim3(kCThreads), lay.total, L.stream, P);
     if (e != cudaSuccess)
         return e;
     note_launches(1);
@@ -681,15 +884,15 @@ cudaError_t cached_launch_ws(const Geom& g, const void* x, const void* M, void* 
 }
 
 template <int WS>
-bool cached_fits(const Geom& g)
+bool cached_fits(const Geom& g, bool fuse)
 {
     CachedLayout lay;
-    return cached_layout<WS>(g, lay);
+    return cached_layout<WS>(g, lay, fuse);
 }
 
 }  // namespace
 
-bool tc_cached_supported(const Geom& g)
+bool tc_cached_supported(const Geom& g, bool fuse)
 {
     if (g.w < 2 || g.w > 15)
         return false;
@@ -698,40 +901,41 @@ bool tc_cached_supported(const Geom& g)
     if (g.bands * (long long)g.C >= (1ll << 31))
         return false;
     switch (g.w) {
-    case 2: return cached_fits<2>(g);
-    case 3: return cached_fits<3>(g);
-    case 4: return cached_fits<4>(g);
-    case 5: return cached_fits<5>(g);
-    case 6: return cached_fits<6>(g);
-    case 7: return cached_fits<7>(g);
-    case 8: return cached_fits<8>(g);
-    case 9: return cached_fits<9>(g);
-    case 10: return cached_fits<10>(g);
-    case 11: return cached_fits<11>(g);
-    case 12: return cached_fits<12>(g);
-    case 13: return cached_fits<13>(g);
-    case 14: return cached_fits<14>(g);
-    default: return cached_fits<15>(g);
+    case 2: return cached_fits<2>(g, fuse);
+    case 3: return cached_fits<3>(g, fuse);
+    case 4: return cached_fits<4>(g, fuse);
+    case 5: return cached_fits<5>(g, fuse);
+    case 6: return cached_fits<6>(g, fuse);
+    case 7: return cached_fits<7>(g, fuse);
+    case 8: return cached_fits<8>(g, fuse);
+    case 9: return cached_fits<9>(g, fuse);
+    case 10: return cached_fits<10>(g, fuse);
+    case 11: return cached_fits<11>(g, fuse);
+    case 12: return cached_fits<12>(g, fuse);
+    case 13: return cached_fits<13>(g, fuse);
+    case 14: return cached_fits<14>(g, fuse);
+    default: return cached_fits<15>(g, fuse);
     }
 }
 
-cudaError_t tc_cached_launch(const Geom& g, const void* x, const void* M, void* y, const Launch& L)
+cudaError_t tc_cached_launch(const Geom& g, const void* x, const void* M, const void* dw, void* y,
+                             const Launch& L)
 {
     switch (g.w) {
-    case 2: return cached_launch_ws<2>(g, x, M, y, L);
-    case 3: return cached_launch_ws<3>(g, x, M, y, L);
-    case 4: return cached_launch_ws<4>(g, x, M, y, L);
-    case 5: return cached_launch_ws<5>(g, x, M, y, L);
-    case 6: return cached_launch_ws<6>(g, x, M, y, L);
-    case 7: return cached_launch_ws<7>(g, x, M, y, L);
-    case 8: return cached_launch_ws<8>(g, x, M, y, L);
-    case 9: return cached_launch_ws<9>(g, x, M, y, L);
-    case 10: return cached_launch_ws<10>(g, x, M, y, L);
-    case 11: return cached_launch_ws<11>(g, x, M, y, L);
-    case 12: return cached_launch_ws<12>(g, x, M, y, L);
-    case 13: return cached_launch_ws<13>(g, x, M, y, L);
-    case 14: return cached_launch_ws<14>(g, x, M, y, L);
-    case 15: return cached_launch_ws<15>(g, x, M, y, L);
+    case 2: return cached_launch_ws<2>(g, x, M, dw, y, L);
+    case 3: return cached_launch_ws<3>(g, x, M, dw, y, L);
+    case 4: return cached_launch_ws<4>(g, x, M, dw, y, L);
+    case 5: return cached_launch_ws<5>(g, x, M, dw, y, L);
+    case 6: return cached_launch_ws<6>(g, x, M, dw, y, L);
+    case 7: return cached_launch_ws<7>(g, x, M, dw, y, L);
+    case 8: return cached_launch_ws<8>(g, x, M, dw, y, L);
+    case 9: return cached_launch_ws<9>(g, x, M, dw, y, L);
+    case 10: return cached_launch_ws<10>(g, x, M, dw, y, L);
+    case 11: return cached_launch_ws<11>(g, x, M, dw, y, L);
+    case 12: return cached_launch_ws<12>(g, x, M, dw, y, L);
+    case 13: return cached_launch_ws<13>(g, x, M, dw, y, L);
+    case 14: return cached_launch_ws<14>(g, x, M, dw, y, L);
+    case 15: return cached_launch_ws<15>(g, x, M, dw, y, L);
     default: return cudaErrorInvalidValue;
     }
 }
