@@ -61,11 +61,14 @@ def test_forward_bf16_small(shape):
     check_bf16(to_np(y), ref, forward_rowbound(xr, Tr, w), "forward")
 
 
-# w = 28 on tensor cores (windows as the MMA's N dimension, a Toeplitz stack
-# of the table as A): one tile of 4 or 15 bands per channel (ragged), three
-# tiles per channel, and enough tiles that CTAs cross channel boundaries and
-# rebuild the stack (checked on sampled channels)
-BIG_SHAPES = [(2, 3, 56, 112, 28), (9, 2, 56, 112, 28), (5, 2, 84, 56, 28), (9, 60, 56, 112, 28)]
+# w = 28 on tensor cores (128 windows per tile as the MMA's M dimension in
+# tensor memory, a Toeplitz stack of the table as B): one partial tile per
+# channel (4, 18 or 15 bands of 32 or 64), one tile on each of 60 CTAs, and
+# three tiles per channel on more tiles than CTAs, so that CTAs take two
+# tiles, cross channel boundaries, rebuild the stack and hand the A rows
+# from one tile to the next (checked on sampled channels)
+BIG_SHAPES = [(2, 3, 56, 112, 28), (9, 2, 56, 112, 28), (5, 2, 84, 56, 28), (9, 60, 56, 112, 28),
+              (40, 60, 56, 112, 28)]
 
 
 @pytest.mark.parametrize("shape", BIG_SHAPES, ids=lambda s: "x".join(map(str, s)))
