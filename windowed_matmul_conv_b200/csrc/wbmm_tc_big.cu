@@ -75,7 +75,7 @@ struct TcBigParams {
     int items;              // C * tpc
     int R;                  // raw ring depth (chunks)
     uint32_t raw_bytes;     // raw chunk slot stride
-    uint32_t off_q, off_raw, off_tst, off_bar;
+    uint32_t off_q, off_raw, off_bar;
     unsigned long long budget;
     int* status;
 };
@@ -98,11 +98,13 @@ __device__ __forceinline__ long long big_row_offset(const TcBigParams& P, int WS
     return (((long long)b * P.C + c) * P.H + (long long)i * WS + row) * P.W;
 }
 
-// Q for one channel from its staged table (K-major, 8-row groups of 256
-// bytes, the two 8-slot core matrices of a row 128 bytes apart).  One thread
-// per (half, row, 8-slot core).
+// Q for one channel from its table Tc in global memory, read reversed for
+// dX (flip) (K-major, 8-row groups of 256 bytes, the two 8-slot core
+// matrices of a row 128 bytes apart).  One thread per (half, row, 8-slot
+// core).
 template <int WS>
-__device__ __forceinline__ void big_build_q(uint8_t* q, const uint16_t* tst, int tid, int nthreads)
+__device__ __forceinline__ void big_build_q(uint8_t* q, const uint16_t* Tc, bool flip, int tid,
+                                            int nthreads)
 {
     using F = BigCfg<WS>;
     for (int item = tid; item < 2 * F::QROWS * 2; item += nthreads) {
@@ -119,8 +121,11 @@ __device__ __forceinline__ void big_build_q(uint8_t* q, const uint16_t* tst, int
             for (int e = 0; e < 2; ++e) {
                 const int s = 16 * h + 8 * core + 2 * m + e;
                 uint16_t v = 0;
-                if (qq < WS && s < WS && dl < F::L)
-                    v = tst[dl * F::L + (qq - s + WS - 1)];
+                if (qq < WS && s < WS && dl < F::L) {
+                    const int e = dl * F::L + (qq - s + WS - 1);
+                    v = __ldg(reinterpret_cast<const unsigned short*>(Tc) +
+                              (flip ? F::TSZ - 1 - e : e));
+                }
                 v2[e] = v;
             }
             wv[m] = pack_bf16x2(v2[0], v2[1]);
@@ -184,7 +189,6 @@ __global__ void __launch_bounds__(kWmThreads, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     uint8_t* q_base = smem + P.off_q;
     uint8_t* raw_base = smem + P.off_raw;
-    uint16_t* tst = reinterpret_cast<uint16_t*>(smem + P.off_tst);
     WmBars& S = *reinterpret_cast<WmBars*>(smem + P.off_bar);
     volatile int* abort = &S.abort;
     const int R = P.R;
@@ -388,16 +392,9 @@ __global__ void __launch_bounds__(kWmThreads, 1)
         constexpr int EPT = kWmEpiWarps * 32;
         const int n = quarter * 32 + lane;
         const uint32_t lanebase = (uint32_t)(quarter * 32) << 16;
-        // Q of channel c.  Every epilogue warp takes part whatever its wait
-        // results, so the named barriers always see all of them.
+        // Q of channel c, built by all epilogue warps; each arrives on q_full.
         auto build_for = [&](int c) {
-            named_bar_sync(2, EPT);                       // staged table fully read
-            const unsigned short* srcT = reinterpret_cast<const unsigned short*>(P.T) +
-                                         (long long)c * F::TSZ;
-            for (int e = et; e < F::TSZ; e += EPT)
-                tst[MODE == kTable ? e : F::TSZ - 1 - e] = __ldg(srcT + e);
-            named_bar_sync(2, EPT);
-            big_build_q<WS>(q_base, tst, et, EPT);
+            big_build_q<WS>(q_base, P.T + (long long)c * F::TSZ, MODE != kTable, et, EPT);
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0)
@@ -457,11 +454,11 @@ __global__ void __launch_bounds__(kWmThreads, 1)
 namespace {
 
 struct BigWmLayout {
-    uint32_t off_q, off_tst, off_bar, off_raw, total, raw_bytes;
+    uint32_t off_q, off_bar, off_raw, total, raw_bytes;
     int R, bpt;
 };
 
-// Q (two halves) | table | barriers | raw ring.
+// Q (two halves) | barriers | raw ring.
 template <int WS>
 bool bigwm_layout(const Geom& g, BigWmLayout& L)
 {
@@ -475,8 +472,6 @@ bool bigwm_layout(const Geom& g, BigWmLayout& L)
     uint32_t off = 0;
     L.off_q = off;
     off += 2 * Q::QH_BYTES;
-    L.off_tst = (off + 15) / 16 * 16;
-    off = L.off_tst + (uint32_t)F::TSZ * 2;
     L.off_bar = (off + 15) / 16 * 16;
     off = L.off_bar + sizeof(WmBars);
     L.off_raw = (off + 127) / 128 * 128;
@@ -519,7 +514,7 @@ cudaError_t bigwm_launch_ws(const Geom& g, const void* x, const void* T, void* y
     P.items = g.C * P.tpc;
     P.R = lay.R;
     P.raw_bytes = lay.raw_bytes;
-    P.off_q = lay.off_q; P.off_raw = lay.off_raw; P.off_tst = lay.off_tst; P.off_bar = lay.off_bar;
+    P.off_q = lay.off_q; P.off_raw = lay.off_raw; P.off_bar = lay.off_bar;
     P.budget = L.budget;
     P.status = L.status;
     int grid = L.num_sms;
