@@ -190,10 +190,12 @@ class ClockSampler:
 class Arm:
     """Device buffers and the step of one workload (one rank)."""
 
-    def __init__(self, wl, seed, nsets, dev):
+    def __init__(self, wl, seed, nsets, dev, fused=False):
         import windowed_matmul_conv_b200 as wb
         self.wb = wb
         self.wl = wl
+        # cached bf16 workloads: the step is the fused cached forward + 3x3
+        self.fused = fused and wl.kind == "cached_dw" and wl.dtype == "bf16"
         self.dev = dev
         d = synth.draw(wl, seed=seed)
         self.host = d
@@ -233,23 +235,26 @@ class Arm:
         if k == "train":
             return ["forward", "backward"]
         if k == "cached_dw":
-            return ["forward_cached", "dw3x3"]
+            return ["forward_cached_dw3x3"] if self.fused else ["forward_cached", "dw3x3"]
         if k == "reparam":
             return ["forward_cached"]
         return ["forward"]
 
     def alternatives(self):
         """Other launches of the same step, timed for reference only: the
-        fused cached forward + 3x3 (one launch; slower on 224x224 planes,
-        where its stencil work blocks the epilogue warps)."""
+        fused cached forward + 3x3 (one launch; slower than the two calls on
+        224x224 planes, where its CUDA-core stencil costs more per tile than
+        the HBM time it saves), or the two calls when --fused makes the
+        fused launch the step."""
         if self.wl.kind == "reparam":
             return ["reparam_merge"]    # one-time preparation of the inference matrix
         if self.wl.kind == "train":
             # one gradient per call: each kernel alone on the whole device
             return ["backward_dx", "backward_dt"]
         # the fused launch covers bf16 maps only
-        return (["forward_cached_dw3x3"] if self.wl.kind == "cached_dw" and self.wl.dtype == "bf16"
-                else [])
+        if self.wl.kind == "cached_dw" and self.wl.dtype == "bf16":
+            return ["forward_cached", "dw3x3"] if self.fused else ["forward_cached_dw3x3"]
+        return []
 
     def calls(self):
         """The step as a user issues it: the training step is one forward
@@ -562,7 +567,7 @@ def run_gpu(args, rank, world, local_rank):
     from windowed_matmul_conv_b200.sharding import channel_range
     peaks = load_peaks()
     peaks["fp32_fma_tflops"] = fp32_fma_peak_tflops(dev)
-    wb_arm = Arm(wl, seed=rank, nsets=3, dev=dev)
+    wb_arm = Arm(wl, seed=rank, nsets=3, dev=dev, fused=args.fused)
     wb = wb_arm.wb
     K, W = args.steps, args.warmup
     stream = torch.cuda.current_stream()
@@ -726,6 +731,8 @@ def run_gpu(args, rank, world, local_rank):
         "kernels": kern,
         "gpu_launches": gpu_launches,
     }
+    if wb_arm.fused:
+        result["config"]["step"] = "fused cached forward + 3x3 (one launch)"
     # roofline of the dominant kernel (HBM-bound at w <= 14: AI ~ d/2 < ridge)
     dom = max(kern, key=lambda n: kern[n]["us"])
     ai = kernel_flops(wl, dom) / kernel_bytes(wl, dom)
@@ -856,6 +863,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-workloads", action="store_true",
                     help="skip the other workloads' timings after the headline step")
+    ap.add_argument("--fused", action="store_true",
+                    help="cached bf16 workloads: time the fused cached forward + 3x3 launch as "
+                         "the step (the two calls become the alternatives)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "wbmm":
         ap.error("at least 3 warm-up steps")
