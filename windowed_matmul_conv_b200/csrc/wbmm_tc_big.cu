@@ -75,6 +75,7 @@ struct TcBigParams {
     int items;              // C * tpc
     int R;                  // raw ring depth (chunks)
     uint32_t raw_bytes;     // raw chunk slot stride
+    uint32_t band_bytes;    // stride of a band's rows in a raw slot (padded)
     uint32_t off_q, off_raw, off_bar;
     unsigned long long budget;
     int* status;
@@ -227,7 +228,8 @@ __global__ void __launch_bounds__(kWmThreads, 1)
     if (warp == 0) {
         // ------------------------------------------------------ producer
         // Chunk ch of tile seq: image rows 4ch .. 4ch+3 of each band of the
-        // tile, band k at slot offset k*CR*W (rows past w are not copied).
+        // tile, band k at slot offset k*band_bytes (rows past w are not
+        // copied).
         int issued = 0;
         bool go = true;
         for (int seq = 0; seq < n_it && go; ++seq) {
@@ -250,7 +252,7 @@ __global__ void __launch_bounds__(kWmThreads, 1)
                     mbar_arrive_expect_tx(&S.raw_full[s], bytes * (uint32_t)t.nb);
                 __syncwarp();
                 for (int k = lane; k < t.nb; k += 32)
-                    bulk_g2s(slot + (size_t)k * F::CR * P.W * 2,
+                    bulk_g2s(slot + (size_t)k * P.band_bytes,
                              P.x + big_row_offset(P, WS, t.c, t.band0 + k, r0), bytes,
                              &S.raw_full[s]);
                 issued = ss + 1;
@@ -360,8 +362,8 @@ __global__ void __launch_bounds__(kWmThreads, 1)
                             break;
                         uint32_t lo[8], hi[8];
                         const uint32_t* src = reinterpret_cast<const uint32_t*>(
-                            raw_base + (size_t)s * P.raw_bytes +
-                            ((size_t)(k * F::CR + rl) * P.W + (size_t)j * WS) * 2);
+                            raw_base + (size_t)s * P.raw_bytes + (size_t)k * P.band_bytes +
+                            ((size_t)rl * P.W + (size_t)j * WS) * 2);
 #pragma unroll
                         for (int m = 0; m < 8; ++m) {
                             lo[m] = (valid && 2 * m < WS) ? src[m] : 0u;
@@ -454,7 +456,7 @@ __global__ void __launch_bounds__(kWmThreads, 1)
 namespace {
 
 struct BigWmLayout {
-    uint32_t off_q, off_bar, off_raw, total, raw_bytes;
+    uint32_t off_q, off_bar, off_raw, total, raw_bytes, band_bytes;
     int R, bpt;
 };
 
@@ -467,7 +469,11 @@ bool bigwm_layout(const Geom& g, BigWmLayout& L)
     if (g.nw < 1 || g.nw > F::NT)
         return false;
     L.bpt = F::NT / g.nw;
-    L.raw_bytes = (uint32_t)L.bpt * F::CR * g.W * 2;
+    // A band's four rows (4*W*2 bytes, a multiple of 64) plus 16 bytes: the
+    // transform's threads (one window each, several bands per warp) then
+    // read shared memory with 2-way instead of 8-way bank conflicts.
+    L.band_bytes = (uint32_t)F::CR * g.W * 2 + 16;
+    L.raw_bytes = (uint32_t)L.bpt * L.band_bytes;
     L.raw_bytes = (L.raw_bytes + 127) / 128 * 128;
     uint32_t off = 0;
     L.off_q = off;
@@ -514,6 +520,7 @@ cudaError_t bigwm_launch_ws(const Geom& g, const void* x, const void* T, void* y
     P.items = g.C * P.tpc;
     P.R = lay.R;
     P.raw_bytes = lay.raw_bytes;
+    P.band_bytes = lay.band_bytes;
     P.off_q = lay.off_q; P.off_raw = lay.off_raw; P.off_bar = lay.off_bar;
     P.budget = L.budget;
     P.status = L.status;
