@@ -417,9 +417,10 @@ __global__ void __launch_bounds__(kDtgMaxThreads, 1)
     const int L = 2 * w - 1, tsz = L * L;
     const int stage_floats = 2 * kCachedNT * DP;  // dY rows, then x rows
     int* colmap = reinterpret_cast<int*>(sgm + 2 * stage_floats);
+    // tile indices fit in 32 bits (the host checks C * ntiles < 2^31)
     const long long G = gridDim.x, Ttot = (long long)C * ntiles;
-    const long long T0 = blockIdx.x * Ttot / G, T1 = (blockIdx.x + 1) * Ttot / G;
-    auto block_of = [&](long long f) { return ((f + 1) * G - 1) / Ttot; };
+    const int T0 = (int)(blockIdx.x * Ttot / G), T1 = (int)((blockIdx.x + 1) * Ttot / G);
+    auto block_of = [&](int f) { return (int)((((long long)f + 1) * G - 1) / Ttot); };
     const int tid = threadIdx.x, nthr = blockDim.x;
     const int lane = tid & 31, warp = tid >> 5, nwarps = nthr >> 5;
     const int ug = tid / VG, vg = tid - (tid / VG) * VG;
@@ -443,23 +444,24 @@ __global__ void __launch_bounds__(kDtgMaxThreads, 1)
     // Tile f (flattened over channels) into stage st: asynchronous copies
     // for fp32 (one commit group per tile), widened through registers for
     // bf16.
-    auto load_tile = [&](long long f, int st) {
+    auto load_tile = [&](int f, int st) {
         float* GS = sgm + (size_t)st * stage_floats;
         float* XS = GS + kCachedNT * DP;
-        const int c = (int)(f / ntiles);
-        const long long g0 = (f - (long long)c * ntiles) * bpt;
-        const int nb = bands - g0 < bpt ? (int)(bands - g0) : bpt;
+        const int c = f / ntiles;
+        const int g0 = (f - c * ntiles) * bpt;                  // bands < 2^31 (host)
+        const int nb = (int)bands - g0 < bpt ? (int)bands - g0 : bpt;
         for (int e = tid; e < (kCachedNT - nb * nw) * DP; e += nthr) {
             GS[nb * nw * DP + e] = 0.0f;
             XS[nb * nw * DP + e] = 0.0f;
         }
         // band kb0 of the tile: image b, band i of that image
-        const long long gb = g0 + kb0;
-        long long b = gb / nh;
-        int i = (int)(gb - b * nh);
+        const int gb = g0 + kb0;
+        int b = gb / nh;
+        int i = gb - b * nh;
         int kb = kb0, r = r0, cu = cu0;
         while (kb < nb) {
-            const long long off = ((b * C + c) * H + (long long)i * w + r) * W + (long long)cu * V;
+            const long long off =
+                ((long long)(b * C + c) * H + i * w + r) * W + (long long)cu * V;
             const int o = kb * nw * DP + r * w + colmap[cu];
             if constexpr (kAsync) {
                 if constexpr (V == 2) {
@@ -504,8 +506,8 @@ __global__ void __launch_bounds__(kDtgMaxThreads, 1)
     int st = 0;
     if (T0 < T1)
         load_tile(T0, 0);
-    for (long long f = T0; f < T1; ++f) {
-        const int c = (int)(f / ntiles);
+    for (int f = T0; f < T1; ++f) {
+        const int c = f / ntiles;
         const bool same_next = f + 1 < T1 && (f + 1) / ntiles == c;
         // stage st ^ 1 was last read by the previous tile, before the barrier
         // that closed its iteration
@@ -587,8 +589,8 @@ __global__ void __launch_bounds__(kDtgMaxThreads, 1)
             }
         }
         __syncthreads();
-        const long long first = block_of((long long)c * ntiles);
-        const int slot = (int)(blockIdx.x - first);
+        const int first = block_of(c * ntiles);
+        const int slot = (int)blockIdx.x - first;
         float* out = part + ((long long)c * S + slot) * tsz;
         for (int bin = tid; bin < tsz; bin += nthr) {
             const int dpi = bin / L, dqi = bin - (bin / L) * L;
@@ -600,7 +602,7 @@ __global__ void __launch_bounds__(kDtgMaxThreads, 1)
             out[bin] = sum;
         }
         if (slot == 0) {
-            const int used = (int)(block_of((long long)c * ntiles + ntiles - 1) - first) + 1;
+            const int used = block_of(c * ntiles + ntiles - 1) - first + 1;
             for (int e = used * tsz + tid; e < S * tsz; e += nthr)
                 part[(long long)c * S * tsz + e] = 0.0f;
         }
@@ -874,12 +876,13 @@ struct DtgPlan {
 bool dtg_plan(const Geom& g, DtgPlan& pl)
 {
     if (g.w < 4 || g.w > 14 || g.nw < 1 || g.nw > kCachedNT || g.bands < 1 || g.C < 1 ||
-        g.nw * g.w > kDtgMaxCols)
+        g.nw * g.w > kDtgMaxCols || g.bands >= (1ll << 31) ||
+        g.bands / g.nh * (long long)g.C >= (1ll << 31))
         return false;
     pl.bpt = kCachedNT / g.nw;
     const long long nt = (g.bands + pl.bpt - 1) / pl.bpt;
     const long long total = nt * g.C;
-    if (nt > (1 << 30) || total > (1ll << 40))
+    if (nt > (1 << 30) || total >= (1ll << 31))
         return false;
     pl.ntiles = (int)nt;
     // blocks resident per SM, by shared memory (233472 bytes per SM, 1 KB
