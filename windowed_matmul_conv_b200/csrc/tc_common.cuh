@@ -66,28 +66,38 @@ __device__ __forceinline__ void band_run(const BandTile& t, const BandRuns& R, i
 
 // Raw band layout -> operand tile with rows = windows n (8-row groups
 // `sbo` bytes apart) and columns = padded positions (core matrices of 8
-// slots, 128 bytes apart).  A warp takes one group of eight windows: lane
-// (nl, rs) handles window 8*g + nl and window rows rs, rs + 4, ...; all of a
-// lane's rows are read before any is written, so its loads overlap.  Eight
-// consecutive lanes take eight consecutive windows, so each quarter-warp
-// store is one contiguous 128-byte line.  Rows nwin <= n < nend are written
-// as zeros; rows past that are left as they are.
+// slots, 128 bytes apart).  A warp takes one group of NWIN windows (8 or
+// 16): lane (nl, rs) = (lane % NWIN, lane / NWIN) handles window NWIN*g + nl
+// and window rows rs, rs + 32/NWIN, ...; all of a lane's rows are read
+// before any is written, so its loads overlap.  Eight consecutive lanes take
+// eight consecutive windows, so each quarter-warp store is one contiguous
+// 128-byte line.  At w = 14, 16 windows x 2 rows per load instruction hit 32
+// different banks for every plane width W = 28k (8 x 4 hit some banks twice);
+// other window sizes keep 8 x 4.  Rows nwin <= n < nend are written as zeros;
+// rows past that are left as they are.
+template <int WS>
+struct TransformCfg {
+    static constexpr int NWIN = WS == 14 ? 16 : 8;      // windows per group
+};
+
 template <int WS>
 __device__ __forceinline__ void transform_group(const uint16_t* raw, uint8_t* dst, uint32_t sbo,
-                                                int g8, int nwin, int nend, const int* woff,
+                                                int gi, int nwin, int nend, const int* woff,
                                                 int W, int lane)
 {
     using P = PadCfg<WS>;
-    constexpr int R4 = (WS + 3) / 4;
-    const int nl = lane & 7, rs = lane >> 3;
-    const int n = g8 * 8 + nl;
+    constexpr int NWIN = TransformCfg<WS>::NWIN;
+    constexpr int NROW = 32 / NWIN;
+    constexpr int RQ = (WS + NROW - 1) / NROW;
+    const int nl = lane % NWIN, rs = lane / NWIN;
+    const int n = gi * NWIN + nl;
     if (n >= nend)
         return;
     const uint16_t* base = raw + woff[n < nwin ? n : 0];
-    uint32_t wv[R4][P::RP / 2];
+    uint32_t wv[RQ][P::RP / 2];
 #pragma unroll
-    for (int q = 0; q < R4; ++q) {
-        const int r = q * 4 + rs;
+    for (int q = 0; q < RQ; ++q) {
+        const int r = q * NROW + rs;
         const uint16_t* src = base + r * W;
         if (n >= nwin || r >= WS) {
 #pragma unroll
@@ -106,10 +116,10 @@ __device__ __forceinline__ void transform_group(const uint16_t* raw, uint8_t* ds
             }
         }
     }
-    uint8_t* d0 = dst + g8 * sbo + nl * 16;
+    uint8_t* d0 = dst + (n >> 3) * sbo + (n & 7) * 16;
 #pragma unroll
-    for (int q = 0; q < R4; ++q) {
-        const int r = q * 4 + rs;
+    for (int q = 0; q < RQ; ++q) {
+        const int r = q * NROW + rs;
         if (r >= WS)
             continue;
 #pragma unroll
@@ -125,11 +135,12 @@ __device__ __forceinline__ void transform_rows(const uint16_t* raw, uint8_t* dst
                                                int nwin, int nzero, const int* woff, int W,
                                                int tid, int nthreads)
 {
+    constexpr int NWIN = TransformCfg<WS>::NWIN;
     const int lane = tid & 31, wid = tid >> 5, nwarps = nthreads >> 5;
     const int nend = nzero > nwin ? nzero : nwin;
-    const int groups = (nend + 7) >> 3;
-    for (int g8 = wid; g8 < groups; g8 += nwarps)
-        transform_group<WS>(raw, dst, sbo, g8, nwin, nend, woff, W, lane);
+    const int groups = (nend + NWIN - 1) / NWIN;
+    for (int gi = wid; gi < groups; gi += nwarps)
+        transform_group<WS>(raw, dst, sbo, gi, nwin, nend, woff, W, lane);
 }
 
 // Two tiles of the same windows (from two tensors) in one pass: warps take
@@ -140,9 +151,10 @@ __device__ __forceinline__ void transform_rows_pair(const uint16_t* raw0, uint8_
                                                     uint32_t sbo, int nwin, int nzero,
                                                     const int* woff, int W, int tid, int nthreads)
 {
+    constexpr int NWIN = TransformCfg<WS>::NWIN;
     const int lane = tid & 31, wid = tid >> 5, nwarps = nthreads >> 5;
     const int nend = nzero > nwin ? nzero : nwin;
-    const int groups = (nend + 7) >> 3;
+    const int groups = (nend + NWIN - 1) / NWIN;
     for (int it = wid; it < 2 * groups; it += nwarps) {
         const bool second = it >= groups;
         transform_group<WS>(second ? raw1 : raw0, second ? dst1 : dst0, sbo,
