@@ -312,12 +312,30 @@ def prefill(ms=20.0):
     torch.cuda._sleep(int(ms * 1e6 * 2.0))   # ~2 GHz cycles per ns
 
 
+def kernel_source_hash(source):
+    """sha256 (16 hex digits) of a kernel source file followed by the local
+    headers it includes (csrc/*.cuh and *.h, in include order), so that a
+    change to shared device code also invalidates a recorded capture."""
+    import hashlib
+    import re
+    path = os.path.join(ROOT, source)
+    h = hashlib.sha256()
+    with open(path, "rb") as f:
+        text = f.read()
+    h.update(text)
+    for inc in re.findall(rb'#include "([^"]+)"', text):
+        hp = os.path.join(os.path.dirname(path), inc.decode())
+        if os.path.exists(hp):
+            with open(hp, "rb") as f:
+                h.update(f.read())
+    return h.hexdigest()[:16]
+
+
 def recorded_traffic(kernel):
     """DRAM bytes per launch from the committed ncu capture, or None when the
     kernel source changed since the counters were taken.  The backward call
     is the sum of its two kernels' captures (ncu runs them one after the
     other, so the second read of dY counts again)."""
-    import hashlib
     if kernel == "backward":
         parts = [recorded_traffic("backward_dx"), recorded_traffic("backward_dt")]
         return None if None in parts else sum(parts)
@@ -326,9 +344,7 @@ def recorded_traffic(kernel):
             rec = json.load(f).get(kernel)
         if not rec:
             return None
-        with open(os.path.join(ROOT, rec["source"]), "rb") as f:
-            sha = hashlib.sha256(f.read()).hexdigest()[:16]
-        return rec["bytes"] if sha == rec["sha256_16"] else None
+        return rec["bytes"] if kernel_source_hash(rec["source"]) == rec["sha256_16"] else None
     except (OSError, ValueError, KeyError):
         return None
 
